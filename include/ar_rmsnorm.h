@@ -1,0 +1,220 @@
+/*
+ * ar_rmsnorm.h -- C ABI of the fused "W-way reduce + residual add + RMSNorm"
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the step that closes a tensor-parallel transformer
+ * sub-layer: the all-reduce of the ranks' partial activations, the residual
+ * add, and RMSNorm.  Here the W partials already sit on one GPU, so the
+ * all-reduce is a W-way elementwise sum done inside the same kernel as the
+ * add and the norm.
+ *
+ * Passages defining the operations (vLLM pull-request reports on
+ * prhub.com.cn; page title, then section):
+ *   - PR #54787 report (ROCm AITER fused allreduce+RMSNorm fast path),
+ *     "关键源码片段": fused_allreduce_gemma_rms_norm returns
+ *     (norm_out, residual_out); its fallback is all_reduce followed by
+ *     GemmaRMSNorm(reduced, residual); gemma_norm selects weight bias 1.0;
+ *     the one-stage predicate is capture-static (depends only on shape,
+ *     dtype and world size).
+ *   - PR #50802 report (AITER add-RMSNorm dead-residual fusion),
+ *     "实现拆解" and "关键源码片段": the output-only pattern keeps only the
+ *     RMSNorm result; the no-residual all_reduce -> rms_norm site; the
+ *     per-group FP8 quantisation of the normalised output, with the bf16
+ *     normalised output also kept for a second consumer.
+ *   - PR #44849 report ([ROCm][MiniMax-M2] fused QK-norm + AllReduce),
+ *     "关键源码片段": _minimax_qk_norm_fusion(qkv, q_weight, k_weight,
+ *     q_size, kv_size, tp_rank, tp_world, eps, ...) normalises q and k over
+ *     their full width across the TP shards.
+ *   - PR #49673 report (token count fix for 3-D inputs), "实现拆解": the
+ *     token count is numel / hidden_dim; here T is passed explicitly and
+ *     callers flatten leading dimensions.
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are caller-owned DEVICE pointers to contiguous
+ *     row-major memory on the current CUDA device.  Pointer arrays
+ *     (`partials`, `qkv`, `q_out`, `k_out`) are HOST arrays of W device
+ *     pointers; they are copied by value into the kernel's parameters, so the
+ *     host array may be reused as soon as the call returns.
+ *   - The library allocates nothing per call, never synchronises, and
+ *     launches on `stream`; calls are asynchronous and may be captured in a
+ *     CUDA graph once the device has been used by one call outside capture
+ *     (the first call on a device reads its attributes and sets kernel
+ *     attributes).
+ *   - Errors are returned synchronously as ar_status and nothing is
+ *     launched; there is no silent no-op and no hidden fallback.  T == 0 is
+ *     valid and launches nothing.  Faults inside a kernel surface as CUDA
+ *     errors on `stream`, as for any kernel.
+ *   - 16-bit formats: AR_BF16 (bfloat16) or AR_FP16 (IEEE half); all 16-bit
+ *     tensors of one call share `dtype`.
+ *   - Accumulation is fp32 with a compensated (error-free transformation)
+ *     sum of the W+1 terms, so r is within one fp32 ulp of the exact sum;
+ *     the sum of squares is combined across threads in fp64; outputs are
+ *     rounded to nearest even.
+ */
+#ifndef AR_RMSNORM_H
+#define AR_RMSNORM_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AR_OK = 0,
+    AR_EINVAL = 1,        /* null required pointer, bad size or count       */
+    AR_EALIGN = 2,        /* a device pointer is not 16-byte aligned         */
+    AR_EUNSUPPORTED = 3,  /* device is not sm_100, or a size beyond limits   */
+    AR_ECUDA = 4,         /* a CUDA runtime call or launch failed            */
+    AR_ETIMEDOUT = 5      /* reserved for bounded device waits               */
+} ar_status;
+
+typedef enum { AR_BF16 = 0, AR_FP16 = 1 } ar_dtype;
+
+/* Largest supported hidden size (elements) and number of partials. */
+#define AR_MAX_H 65536
+#define AR_MAX_W 16
+
+/*
+ * ar_add_rmsnorm -- two-output, output-only and no-residual forms.
+ *
+ *   r[t,h] = residual[t,h] + sum_{w<W} partials[w][t,h]
+ *   y[t,h] = r[t,h] * rsqrt(mean_h(r[t,:]^2) + eps) * (gemma ? 1 + weight[h]
+ *                                                          : weight[h])
+ *   out[t,h]          = RNE_dtype(y[t,h])
+ *   residual_out[t,h] = RNE_dtype(r[t,h])
+ *
+ * partials      host array of W device pointers, each [T, H] in `dtype`
+ * residual      [T, H] or NULL (NULL: r is the plain sum, the no-residual
+ *               form all_reduce -> rms_norm)
+ * weight        [H]
+ * out           [T, H], written
+ * residual_out  [T, H] or NULL (NULL: the dead-residual / output-only form;
+ *               nothing is written).  residual_out == residual (in place) is
+ *               allowed; any other overlap between outputs and inputs is
+ *               undefined.
+ * T             tokens (rows), >= 0
+ * H             hidden size, multiple of 8, 8 <= H <= AR_MAX_H
+ * W             number of partials, 1 <= W <= AR_MAX_W
+ * eps           finite, >= 0; added to the mean of squares inside the rsqrt
+ * gemma         0: weight w;  1: weight (1 + w), the Gemma RMSNorm variant
+ * dtype         AR_BF16 or AR_FP16
+ * Alignment: every pointer 16-byte aligned (AR_EALIGN otherwise).
+ */
+int ar_add_rmsnorm(const void *const *partials, const void *residual,
+                   const void *weight, void *out, void *residual_out,
+                   int64_t T, int64_t H, int W, float eps, int gemma,
+                   int dtype, cudaStream_t stream);
+
+/*
+ * ar_add_rmsnorm_quant_fp8_group -- the same r and y, then per-group FP8.
+ * (PR #50802 report: all_reduce -> add -> RMSNorm -> per-group FP8 quant,
+ * with the 16-bit normalised output kept for a second consumer.)
+ *
+ * For each group g of `group` consecutive elements of a row, with y in fp32:
+ *   amax          = max |y| over the group
+ *   scales[t,g]   = amax / 448                  (IEEE fp32 division)
+ *   out_fp8[t,h]  = e4m3fn_RNE_satfinite(y[t,h] / scales[t,g]),
+ *                   0 for every element when amax == 0
+ * out_fp8       [T, H] bytes, OCP e4m3fn codes (1-4-3, bias 7, max 448)
+ * scales        [T, H/group] fp32, row-major
+ * out_y         [T, H] in `dtype` (RNE of y) or NULL
+ * residual_out  [T, H] in `dtype` or NULL, as in ar_add_rmsnorm
+ * group         must be 128; H must be a multiple of it
+ * Other arguments as in ar_add_rmsnorm.  scales needs 4-byte alignment, all
+ * other pointers 16-byte alignment.
+ */
+int ar_add_rmsnorm_quant_fp8_group(const void *const *partials,
+                                   const void *residual, const void *weight,
+                                   void *out_fp8, float *scales, void *out_y,
+                                   void *residual_out, int64_t T, int64_t H,
+                                   int W, int group, float eps, int gemma,
+                                   int dtype, cudaStream_t stream);
+
+/*
+ * qk_norm_sharded -- MiniMax-style QK-norm over W tensor-parallel shards.
+ * (PR #44849 report: q and k of each shard are normalised over the full
+ * q (k) width; the only cross-shard quantity is a token's sum of squares.)
+ *
+ * qs = q_size / W, ks = kv_size / W.  Shard w's buffer qkv[w] is [T, qs+2ks]
+ * with row layout [ q_w | k_w | v_w ].  For each token t:
+ *   inv_q = rsqrt(sum_{w,j} q_w[t,j]^2 / q_size + eps)
+ *   inv_k = rsqrt(sum_{w,j} k_w[t,j]^2 / kv_size + eps)
+ *   q_out[w][t,j] = RNE(q_w[t,j] * inv_q * q_weight[w*qs + j])
+ *   k_out[w][t,j] = RNE(k_w[t,j] * inv_k * k_weight[w*ks + j])
+ * v is neither read nor written.
+ *
+ * qkv       host array of W device pointers, each [T, qs + 2*ks]
+ * q_weight  [q_size];  k_weight [kv_size]  (full vectors; shard w uses its
+ *           slice)
+ * q_out     host array of W device pointers, each [T, qs], dense
+ * k_out     host array of W device pointers, each [T, ks], dense
+ * Requirements: 1 <= W <= AR_MAX_W, q_size and kv_size positive multiples
+ * of W with qs and ks multiples of 8, qs + ks <= AR_MAX_H, pointers 16-byte
+ * aligned, outputs not overlapping inputs.
+ */
+int qk_norm_sharded(const void *const *qkv, const void *q_weight,
+                    const void *k_weight, void *const *q_out,
+                    void *const *k_out, int64_t T, int64_t q_size,
+                    int64_t kv_size, int W, float eps, int dtype,
+                    cudaStream_t stream);
+
+/*
+ * Dispatch plans.  Each call picks a kernel configuration ("plan") from a
+ * table of measured timings keyed by (variant, dtype, W, H, T range), and
+ * falls back to a built-in rule for shapes the table does not cover.  The
+ * choice depends only on these arguments and the loaded table, never on
+ * data or device state, so it is the same during CUDA-graph capture as
+ * outside it (the PR #54787 report's "capture-static" property).
+ */
+typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_variant;
+
+/* Plan ids.  ROWC<k>: one row per cluster of k CTAs (sum of squares combined
+ * through distributed shared memory).  PERSIST: one CTA per row, grid sized
+ * to the SM count, rows looped.  BULK: PERSIST with rows staged into shared
+ * memory by bulk asynchronous copies.  QK_C<k>: one token per cluster of k
+ * CTAs, shards split across the cluster. */
+enum {
+    AR_PLAN_AUTO = 0,
+    AR_PLAN_ROWC1 = 1,
+    AR_PLAN_ROWC2 = 2,
+    AR_PLAN_ROWC4 = 3,
+    AR_PLAN_ROWC8 = 4,
+    AR_PLAN_PERSIST = 5,
+    AR_PLAN_BULK = 6,
+    AR_PLAN_QK_C1 = 11,
+    AR_PLAN_QK_C2 = 12,
+    AR_PLAN_QK_C4 = 13,
+    AR_PLAN_QK_C8 = 14
+};
+
+/* The plan a call with these arguments would use (for QK, H = q_size + kv_size
+ * per token, W the shard count).  Writes *plan_id; returns AR_EINVAL for a bad
+ * variant, dtype or null plan_id. */
+int ar_plan_query(int variant, int64_t T, int64_t H, int W, int dtype,
+                  int *plan_id);
+
+/* Load a plan table (JSON: {"entries": [{"variant":v, "dtype":d, "W":w,
+ * "H":h, "t_lo":a, "t_hi":b, "plan":p}, ...]}).  The table replaces the
+ * loaded one only if the whole file parses and every plan id is valid for
+ * its variant; otherwise AR_EINVAL is returned and the previous table stays.
+ * path == NULL clears the table (built-in rule only).  Not safe to call
+ * concurrently with launches on other threads. */
+int ar_plan_load(const char *path);
+
+/* Force `plan_id` for every call of `variant` (AR_PLAN_AUTO clears).  For A/B
+ * measurement; AR_EINVAL for an id that does not belong to the variant. */
+int ar_plan_force(int variant, int plan_id);
+
+/* Number of table entries currently loaded. */
+int ar_plan_table_size(void);
+
+/* Static description of a status code. */
+const char *ar_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AR_RMSNORM_H */

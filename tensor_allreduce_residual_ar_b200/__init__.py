@@ -1,0 +1,10 @@
+"""Fused W-way reduce + residual add + RMSNorm for NVIDIA B200 (sm_100a).
+
+The compute lives in a C-ABI CUDA library (``csrc/``, header
+``include/ar_rmsnorm.h``); this package is its thin Python binding.
+"""
+from .binding import (  # noqa: F401
+    AR_BF16, AR_FP16, ARError, ar_add_rmsnorm, ar_add_rmsnorm_quant_fp8_group,
+    ar_plan_force, ar_plan_load, ar_plan_query, ar_plan_table_size, ar_status_string,
+    library_path, load_library, qk_norm_sharded,
+)

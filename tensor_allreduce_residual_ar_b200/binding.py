@@ -1,0 +1,171 @@
+"""ctypes binding of the C ABI in ``include/ar_rmsnorm.h``.
+
+Argument marshalling only: shapes, dtypes and device pointers are read from
+torch tensors and handed to the C entry points of the same names, on torch's
+current CUDA stream unless a stream is given.  Every step of the computation
+runs in the library's CUDA kernels; there is no Python or CPU fallback, and a
+missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+AR_BF16 = 0
+AR_FP16 = 1
+_DTYPES = {torch.bfloat16: AR_BF16, torch.float16: AR_FP16}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "_lib", "libar_rmsnorm.so")
+_PLAN_TABLE = os.path.join(_HERE, "plan_table.json")
+_lock = threading.Lock()
+_lib = None
+
+
+class ARError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {ar_status_string(status)} (status {status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load the CUDA library (built by ``tensor_allreduce_residual_ar_b200.build``)
+    and its shipped plan table.  Raises if the library is missing."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library not built: {_LIB_PATH} is missing; run "
+                "`python -c 'import __graft_entry__ as g; g.build()'` first")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        PP = ctypes.POINTER(ctypes.c_void_p)
+        lib.ar_add_rmsnorm.restype = i32
+        lib.ar_add_rmsnorm.argtypes = [PP, P, P, P, P, i64, i64, i32, f32, i32, i32, P]
+        lib.ar_add_rmsnorm_quant_fp8_group.restype = i32
+        lib.ar_add_rmsnorm_quant_fp8_group.argtypes = [PP, P, P, P, P, P, P, i64, i64, i32, i32,
+                                                       f32, i32, i32, P]
+        lib.qk_norm_sharded.restype = i32
+        lib.qk_norm_sharded.argtypes = [PP, P, P, PP, PP, i64, i64, i64, i32, f32, i32, P]
+        lib.ar_plan_query.restype = i32
+        lib.ar_plan_query.argtypes = [i32, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_int)]
+        lib.ar_plan_load.restype = i32
+        lib.ar_plan_load.argtypes = [ctypes.c_char_p]
+        lib.ar_plan_force.restype = i32
+        lib.ar_plan_force.argtypes = [i32, i32]
+        lib.ar_plan_table_size.restype = i32
+        lib.ar_plan_table_size.argtypes = []
+        lib.ar_status_string.restype = ctypes.c_char_p
+        lib.ar_status_string.argtypes = [i32]
+        if os.path.exists(_PLAN_TABLE):
+            st = lib.ar_plan_load(_PLAN_TABLE.encode())
+            if st != 0:
+                raise RuntimeError(f"shipped plan table {_PLAN_TABLE} rejected (status {st})")
+        _lib = lib
+        return lib
+
+
+def ar_status_string(status: int) -> str:
+    return load_library().ar_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise ARError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _ptrs(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float16") from None
+
+
+def _rows(t: torch.Tensor, H: int) -> int:
+    """Token count of a [..., H] tensor: numel // H (leading dims flattened)."""
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    if t.shape[-1] != H:
+        raise ValueError(f"last dimension {t.shape[-1]} != {H}")
+    return t.numel() // H
+
+
+def ar_add_rmsnorm(partials, residual, weight, out, residual_out=None, eps: float = 1e-6,
+                   gemma: bool = False, stream=None) -> None:
+    """out = RMSNorm(residual + sum(partials)) * weight (or 1 + weight);
+    residual_out = residual + sum(partials).  ``residual`` and
+    ``residual_out`` may be None.  All tensors [..., H] on one CUDA device."""
+    H = weight.shape[-1]
+    T = _rows(partials[0], H)
+    lib = load_library()
+    _check("ar_add_rmsnorm", lib.ar_add_rmsnorm(
+        _ptrs(partials), _ptr(residual), _ptr(weight), _ptr(out), _ptr(residual_out),
+        T, H, len(partials), float(eps), int(bool(gemma)), _dtype(weight), _stream(stream)))
+
+
+def ar_add_rmsnorm_quant_fp8_group(partials, residual, weight, out_fp8, scales, out_y=None,
+                                   residual_out=None, eps: float = 1e-6, gemma: bool = False,
+                                   group: int = 128, stream=None) -> None:
+    """As ar_add_rmsnorm, then per-group e4m3 codes ``out_fp8`` (uint8 or
+    float8_e4m3fn [..., H]) and fp32 ``scales`` [..., H/group]; the 16-bit y
+    goes to ``out_y`` when given."""
+    H = weight.shape[-1]
+    T = _rows(partials[0], H)
+    lib = load_library()
+    _check("ar_add_rmsnorm_quant_fp8_group", lib.ar_add_rmsnorm_quant_fp8_group(
+        _ptrs(partials), _ptr(residual), _ptr(weight), _ptr(out_fp8), _ptr(scales), _ptr(out_y),
+        _ptr(residual_out), T, H, len(partials), int(group), float(eps), int(bool(gemma)),
+        _dtype(weight), _stream(stream)))
+
+
+def qk_norm_sharded(qkv, q_weight, k_weight, q_out, k_out, q_size: int, kv_size: int,
+                    eps: float = 1e-6, stream=None) -> None:
+    """Sharded QK-norm over W = len(qkv) shards, each [T, q_size/W + 2*kv_size/W]."""
+    W = len(qkv)
+    row = q_size // W + 2 * (kv_size // W)
+    T = _rows(qkv[0], row)
+    lib = load_library()
+    _check("qk_norm_sharded", lib.qk_norm_sharded(
+        _ptrs(qkv), _ptr(q_weight), _ptr(k_weight), _ptrs(q_out), _ptrs(k_out), T, int(q_size),
+        int(kv_size), W, float(eps), _dtype(q_weight), _stream(stream)))
+
+
+def ar_plan_query(variant: int, T: int, H: int, W: int, dtype: int) -> int:
+    pid = ctypes.c_int(-1)
+    _check("ar_plan_query", load_library().ar_plan_query(variant, T, H, W, dtype, ctypes.byref(pid)))
+    return pid.value
+
+
+def ar_plan_load(path) -> int:
+    return load_library().ar_plan_load(None if path is None else str(path).encode())
+
+
+def ar_plan_force(variant: int, plan_id: int) -> int:
+    return load_library().ar_plan_force(variant, plan_id)
+
+
+def ar_plan_table_size() -> int:
+    return load_library().ar_plan_table_size()

@@ -1,0 +1,35 @@
+"""Shared pytest configuration.
+
+Markers:
+  gpu  -- needs a CUDA device (B200, sm_100a); run with ``-m gpu``.
+Everything unmarked runs on a CPU-only host.
+"""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a)")
+
+
+@pytest.fixture(scope="session")
+def cuda_device():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device on this host")
+    return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def lib(cuda_device):
+    """The CUDA library through its Python binding.  On a GPU host a missing
+    or unloadable library is an error, never a skip."""
+    import tensor_allreduce_residual_ar_b200 as ar
+    ar.load_library()
+    return ar
