@@ -57,6 +57,12 @@
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
+#if defined(__GNUC__)
+#define AR_API __attribute__((visibility("default")))
+#else
+#define AR_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -102,7 +108,7 @@ typedef enum { AR_BF16 = 0, AR_FP16 = 1 } ar_dtype;
  * dtype         AR_BF16 or AR_FP16
  * Alignment: every pointer 16-byte aligned (AR_EALIGN otherwise).
  */
-int ar_add_rmsnorm(const void *const *partials, const void *residual,
+AR_API int ar_add_rmsnorm(const void *const *partials, const void *residual,
                    const void *weight, void *out, void *residual_out,
                    int64_t T, int64_t H, int W, float eps, int gemma,
                    int dtype, cudaStream_t stream);
@@ -125,7 +131,7 @@ int ar_add_rmsnorm(const void *const *partials, const void *residual,
  * Other arguments as in ar_add_rmsnorm.  scales needs 4-byte alignment, all
  * other pointers 16-byte alignment.
  */
-int ar_add_rmsnorm_quant_fp8_group(const void *const *partials,
+AR_API int ar_add_rmsnorm_quant_fp8_group(const void *const *partials,
                                    const void *residual, const void *weight,
                                    void *out_fp8, float *scales, void *out_y,
                                    void *residual_out, int64_t T, int64_t H,
@@ -154,7 +160,7 @@ int ar_add_rmsnorm_quant_fp8_group(const void *const *partials,
  * of W with qs and ks multiples of 8, qs + ks <= AR_MAX_H, pointers 16-byte
  * aligned, outputs not overlapping inputs.
  */
-int qk_norm_sharded(const void *const *qkv, const void *q_weight,
+AR_API int qk_norm_sharded(const void *const *qkv, const void *q_weight,
                     const void *k_weight, void *const *q_out,
                     void *const *k_out, int64_t T, int64_t q_size,
                     int64_t kv_size, int W, float eps, int dtype,
@@ -192,7 +198,7 @@ enum {
 /* The plan a call with these arguments would use (for QK, H = q_size + kv_size
  * per token, W the shard count).  Writes *plan_id; returns AR_EINVAL for a bad
  * variant, dtype or null plan_id. */
-int ar_plan_query(int variant, int64_t T, int64_t H, int W, int dtype,
+AR_API int ar_plan_query(int variant, int64_t T, int64_t H, int W, int dtype,
                   int *plan_id);
 
 /* Load a plan table (JSON: {"entries": [{"variant":v, "dtype":d, "W":w,
@@ -201,17 +207,17 @@ int ar_plan_query(int variant, int64_t T, int64_t H, int W, int dtype,
  * its variant; otherwise AR_EINVAL is returned and the previous table stays.
  * path == NULL clears the table (built-in rule only).  Not safe to call
  * concurrently with launches on other threads. */
-int ar_plan_load(const char *path);
+AR_API int ar_plan_load(const char *path);
 
 /* Force `plan_id` for every call of `variant` (AR_PLAN_AUTO clears).  For A/B
  * measurement; AR_EINVAL for an id that does not belong to the variant. */
-int ar_plan_force(int variant, int plan_id);
+AR_API int ar_plan_force(int variant, int plan_id);
 
 /* Number of table entries currently loaded. */
-int ar_plan_table_size(void);
+AR_API int ar_plan_table_size(void);
 
 /* Static description of a status code. */
-const char *ar_status_string(int status);
+AR_API const char *ar_status_string(int status);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,346 @@
+// ar_rmsnorm.cu -- C ABI entry points: argument validation, plan dispatch,
+// launch geometry and kernel launch on the caller's stream.
+//
+// Error behaviour follows two lessons of the vLLM reports: never a silent
+// no-op on an unsupported size (PR #54787 report, section 风险与影响, item 1),
+// and no try/except-style fallback that hides a failure (PR #44849 report,
+// section 评论区精华).  Every rejection is a status code, and nothing is
+// launched after a rejection.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "ar_rmsnorm.h"
+#include "kernels.cuh"
+#include "plan.h"
+
+using namespace arn;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DevInfo {
+    int sm_count = 0;
+    int status = AR_OK;
+};
+
+DevInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+// Device facts, read once per device.  sm_100a code runs only on compute
+// capability 10.0 (B200); anything else is AR_EUNSUPPORTED.
+int device_info(DevInfo &out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return AR_ECUDA;
+    if (dev < 0 || dev >= kMaxDevices) return AR_EUNSUPPORTED;
+    std::call_once(g_dev_once[dev], [dev] {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            g_dev[dev].status = AR_ECUDA;
+            return;
+        }
+        g_dev[dev].status = (major == 10 && minor == 0) ? AR_OK : AR_EUNSUPPORTED;
+        g_dev[dev].sm_count = sms;
+    });
+    out = g_dev[dev];
+    return out.status;
+}
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+constexpr int kPptVariants = 3;   // packs per thread 1, 2, 4
+
+int wb_bucket(int W) { return W <= 2 ? 0 : W <= 4 ? 1 : W <= 8 ? 2 : 3; }   // 2, 4, 8, 16
+
+// ---------------------------------------------------------------------------
+// launch tables
+// ---------------------------------------------------------------------------
+
+using NormKernel = void (*)(const NormParams);
+using QKKernel = void (*)(const QKParams);
+
+template <typename Elt, bool FP8>
+NormKernel norm_kernel_for(int wb, int ppt_idx) {
+#define ARN_K(WB, PPT) &norm_rows_kernel<Elt, WB, PPT, FP8>
+    static const NormKernel tab[4][kPptVariants] = {
+        {ARN_K(2, 1), ARN_K(2, 2), ARN_K(2, 4)},
+        {ARN_K(4, 1), ARN_K(4, 2), ARN_K(4, 4)},
+        {ARN_K(8, 1), ARN_K(8, 2), ARN_K(8, 4)},
+        {ARN_K(16, 1), ARN_K(16, 2), ARN_K(16, 4)},
+    };
+#undef ARN_K
+    return tab[wb][ppt_idx];
+}
+
+NormKernel pick_norm_kernel(int dtype, bool fp8, int wb, int ppt_idx) {
+    if (dtype == AR_BF16)
+        return fp8 ? norm_kernel_for<__nv_bfloat16, true>(wb, ppt_idx)
+                   : norm_kernel_for<__nv_bfloat16, false>(wb, ppt_idx);
+    return fp8 ? norm_kernel_for<__half, true>(wb, ppt_idx) : norm_kernel_for<__half, false>(wb, ppt_idx);
+}
+
+QKKernel pick_qk_kernel(int dtype, int ppt_idx) {
+    static const QKKernel bf[kPptVariants] = {&qk_norm_kernel<__nv_bfloat16, 1>,
+                                              &qk_norm_kernel<__nv_bfloat16, 2>,
+                                              &qk_norm_kernel<__nv_bfloat16, 4>};
+    static const QKKernel hf[kPptVariants] = {&qk_norm_kernel<__half, 1>, &qk_norm_kernel<__half, 2>,
+                                              &qk_norm_kernel<__half, 4>};
+    return dtype == AR_BF16 ? bf[ppt_idx] : hf[ppt_idx];
+}
+
+// Threads per CTA and packs per thread for `packs` packs per CTA: the
+// fewest packs per thread (1, 2, 4) that fit within max_threads.
+bool split_threads(int packs, int max_threads, int &threads, int &ppt_idx) {
+    for (int i = 0; i < kPptVariants; ++i) {
+        const int ppt = 1 << i;
+        const int t = (packs + ppt - 1) / ppt;
+        if (t <= max_threads) {
+            threads = ((t + 31) / 32) * 32;
+            ppt_idx = i;
+            return true;
+        }
+    }
+    return false;
+}
+
+// Occupancy (resident CTAs per SM) of a kernel at a block size, cached.
+struct OccKey { const void *fn; int threads; int dev; };
+struct OccSlot { OccKey key; int occ; };
+std::mutex g_occ_mutex;
+OccSlot g_occ[256];
+int g_occ_n = 0;
+
+int occupancy(const void *fn, int threads, int dev) {
+    std::lock_guard<std::mutex> lk(g_occ_mutex);
+    for (int i = 0; i < g_occ_n; ++i)
+        if (g_occ[i].key.fn == fn && g_occ[i].key.threads == threads && g_occ[i].key.dev == dev)
+            return g_occ[i].occ;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, 0) != cudaSuccess || occ < 1)
+        occ = 1;
+    if (g_occ_n < 256) g_occ[g_occ_n++] = {{fn, threads, dev}, occ};
+    return occ;
+}
+
+template <typename Params>
+int launch(void (*fn)(const Params), const Params &p, int64_t clusters, int C, int threads,
+           cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(clusters * C), 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (C > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, fn, p) == cudaSuccess ? AR_OK : AR_ECUDA;
+}
+
+// Grid size in clusters: one per row, or capped for persistent plans.
+int64_t grid_clusters(int64_t rows, const Geometry &g, const void *fn, int threads, int dev,
+                      int sm_count) {
+    int64_t cap = (int64_t)0x7FFFFFFF / g.C;
+    if (g.persistent) cap = (int64_t)sm_count * occupancy(fn, threads, dev) / g.C;
+    if (cap < 1) cap = 1;
+    return rows < cap ? rows : cap;
+}
+
+int validate_norm_common(const void *const *partials, const void *residual, const void *weight,
+                         void *residual_out, int64_t T, int64_t H, int W, float eps, int dtype) {
+    if (partials == nullptr || weight == nullptr) return AR_EINVAL;
+    if (W < 1 || W > AR_MAX_W) return AR_EINVAL;
+    if (T < 0 || H < 8 || H % 8 != 0) return AR_EINVAL;
+    if (H > AR_MAX_H) return AR_EUNSUPPORTED;
+    if (dtype != AR_BF16 && dtype != AR_FP16) return AR_EINVAL;
+    if (!std::isfinite(eps) || eps < 0.f) return AR_EINVAL;
+    for (int w = 0; w < W; ++w) {
+        if (partials[w] == nullptr) return AR_EINVAL;
+        if (!aligned(partials[w], 16)) return AR_EALIGN;
+    }
+    if (!aligned(weight, 16)) return AR_EALIGN;
+    if (residual && !aligned(residual, 16)) return AR_EALIGN;
+    if (residual_out && !aligned(residual_out, 16)) return AR_EALIGN;
+    return AR_OK;
+}
+
+int run_norm(const void *const *partials, const void *residual, const void *weight, void *out,
+             void *residual_out, uint8_t *out_fp8, float *scales, int64_t T, int64_t H, int W,
+             float eps, int gemma, int dtype, bool fp8, cudaStream_t stream) {
+    DevInfo di;
+    int st = device_info(di);
+    if (st != AR_OK) return st;
+    int dev = 0;
+    cudaGetDevice(&dev);
+
+    NormParams p = {};
+    for (int w = 0; w < W; ++w) p.partials[w] = partials[w];
+    p.residual = residual;
+    p.weight = weight;
+    p.out = out;
+    p.residual_out = residual_out;
+    p.out_fp8 = out_fp8;
+    p.scales = scales;
+    p.T = T;
+    p.P = (int)(H / 8);
+    p.W = W;
+    p.inv_H = 1.0 / (double)H;
+    p.eps = (double)eps;
+    p.gemma = gemma ? 1 : 0;
+
+    const int variant = fp8 ? AR_VARIANT_FP8 : AR_VARIANT_NORM;
+    const int plan = plan_lookup(variant, T, H, W, dtype, di.sm_count);
+    Geometry g = plan_geometry(plan);
+    // never split a row into slices narrower than one FP8 group
+    while (g.C > 1 && (p.P + g.C - 1) / g.C < kGroupPacks) g.C /= 2;
+    int ppc = 0, threads = 0, ppt_idx = 0;
+    for (;;) {
+        ppc = (p.P + g.C - 1) / g.C;
+        if (fp8) ppc = ((ppc + kGroupPacks - 1) / kGroupPacks) * kGroupPacks;
+        if (split_threads(ppc, g.max_threads, threads, ppt_idx) ||
+            split_threads(ppc, kMaxThreads, threads, ppt_idx))
+            break;
+        // a row too wide for this plan's cluster: widen the cluster
+        if (g.C >= 8) return AR_EUNSUPPORTED;
+        g.C *= 2;
+        g.persistent = false;
+    }
+    p.C = g.C;
+    p.ppc = ppc;
+    NormKernel fn = pick_norm_kernel(dtype, fp8, wb_bucket(W), ppt_idx);
+    const int64_t clusters = grid_clusters(T, g, (const void *)fn, threads, dev, di.sm_count);
+    return launch(fn, p, clusters, g.C, threads, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ar_add_rmsnorm(const void *const *partials, const void *residual, const void *weight, void *out,
+                   void *residual_out, int64_t T, int64_t H, int W, float eps, int gemma, int dtype,
+                   cudaStream_t stream) {
+    int st = validate_norm_common(partials, residual, weight, residual_out, T, H, W, eps, dtype);
+    if (st != AR_OK) return st;
+    if (out == nullptr) return AR_EINVAL;
+    if (!aligned(out, 16)) return AR_EALIGN;
+    if (T == 0) return AR_OK;
+    return run_norm(partials, residual, weight, out, residual_out, nullptr, nullptr, T, H, W, eps,
+                    gemma, dtype, false, stream);
+}
+
+int ar_add_rmsnorm_quant_fp8_group(const void *const *partials, const void *residual,
+                                   const void *weight, void *out_fp8, float *scales, void *out_y,
+                                   void *residual_out, int64_t T, int64_t H, int W, int group,
+                                   float eps, int gemma, int dtype, cudaStream_t stream) {
+    int st = validate_norm_common(partials, residual, weight, residual_out, T, H, W, eps, dtype);
+    if (st != AR_OK) return st;
+    if (out_fp8 == nullptr || scales == nullptr) return AR_EINVAL;
+    if (group != 128 || H % group != 0) return AR_EINVAL;
+    if (!aligned(out_fp8, 16) || !aligned(scales, 4)) return AR_EALIGN;
+    if (out_y && !aligned(out_y, 16)) return AR_EALIGN;
+    if (T == 0) return AR_OK;
+    return run_norm(partials, residual, weight, out_y, residual_out, (uint8_t *)out_fp8, scales, T, H,
+                    W, eps, gemma, dtype, true, stream);
+}
+
+int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_weight,
+                    void *const *q_out, void *const *k_out, int64_t T, int64_t q_size,
+                    int64_t kv_size, int W, float eps, int dtype, cudaStream_t stream) {
+    if (qkv == nullptr || q_out == nullptr || k_out == nullptr || q_weight == nullptr ||
+        k_weight == nullptr)
+        return AR_EINVAL;
+    if (W < 1 || W > AR_MAX_W || T < 0) return AR_EINVAL;
+    if (q_size <= 0 || kv_size <= 0 || q_size % W != 0 || kv_size % W != 0) return AR_EINVAL;
+    const int64_t qs = q_size / W, ks = kv_size / W;
+    if (qs % 8 != 0 || ks % 8 != 0) return AR_EINVAL;
+    if (qs + ks > AR_MAX_H) return AR_EUNSUPPORTED;
+    if (dtype != AR_BF16 && dtype != AR_FP16) return AR_EINVAL;
+    if (!std::isfinite(eps) || eps < 0.f) return AR_EINVAL;
+    for (int w = 0; w < W; ++w) {
+        if (qkv[w] == nullptr || q_out[w] == nullptr || k_out[w] == nullptr) return AR_EINVAL;
+        if (!aligned(qkv[w], 16) || !aligned(q_out[w], 16) || !aligned(k_out[w], 16)) return AR_EALIGN;
+    }
+    if (!aligned(q_weight, 16) || !aligned(k_weight, 16)) return AR_EALIGN;
+    if (T == 0) return AR_OK;
+
+    DevInfo di;
+    int st = device_info(di);
+    if (st != AR_OK) return st;
+    int dev = 0;
+    cudaGetDevice(&dev);
+
+    QKParams p = {};
+    for (int w = 0; w < W; ++w) {
+        p.qkv[w] = qkv[w];
+        p.q_out[w] = q_out[w];
+        p.k_out[w] = k_out[w];
+    }
+    p.q_weight = q_weight;
+    p.k_weight = k_weight;
+    p.T = T;
+    p.W = W;
+    p.qsp = (int)(qs / 8);
+    p.ksp = (int)(ks / 8);
+    p.row_packs = p.qsp + 2 * p.ksp;
+    p.inv_q = 1.0 / (double)q_size;
+    p.inv_k = 1.0 / (double)kv_size;
+    p.eps = (double)eps;
+
+    const int plan = plan_lookup(AR_VARIANT_QK, T, q_size + kv_size, W, dtype, di.sm_count);
+    Geometry g = plan_geometry(plan);
+    while (g.C > 1 && W % g.C != 0) g.C /= 2;
+    int threads = 0, ppt_idx = 0;
+    for (;;) {
+        p.spc = W / g.C;
+        const int npk = p.spc * (p.qsp + p.ksp);
+        if (split_threads(npk, g.max_threads, threads, ppt_idx) ||
+            split_threads(npk, kMaxThreads, threads, ppt_idx))
+            break;
+        // a token too wide for this plan's cluster: split it over more CTAs
+        if (g.C >= 8 || W % (2 * g.C) != 0) return AR_EUNSUPPORTED;
+        g.C *= 2;
+    }
+    p.C = g.C;
+    QKKernel fn = pick_qk_kernel(dtype, ppt_idx);
+    const int64_t clusters = grid_clusters(T, g, (const void *)fn, threads, dev, di.sm_count);
+    return launch(fn, p, clusters, g.C, threads, stream);
+}
+
+int ar_plan_query(int variant, int64_t T, int64_t H, int W, int dtype, int *plan_id) {
+    if (plan_id == nullptr || variant < 0 || variant > 2) return AR_EINVAL;
+    if (dtype != AR_BF16 && dtype != AR_FP16) return AR_EINVAL;
+    if (W < 1 || W > AR_MAX_W || T < 0 || H < 8) return AR_EINVAL;
+    int sms = 148;
+    DevInfo di;
+    if (device_info(di) == AR_OK) sms = di.sm_count;
+    *plan_id = plan_lookup(variant, T, H, W, dtype, sms);
+    return AR_OK;
+}
+
+int ar_plan_load(const char *path) { return plan_load_file(path); }
+
+int ar_plan_force(int variant, int plan_id) { return plan_force(variant, plan_id); }
+
+int ar_plan_table_size(void) { return plan_table_size(); }
+
+const char *ar_status_string(int status) {
+    switch (status) {
+    case AR_OK: return "AR_OK: success";
+    case AR_EINVAL: return "AR_EINVAL: invalid argument (null pointer, size or count)";
+    case AR_EALIGN: return "AR_EALIGN: pointer not aligned (16 bytes; 4 for scales)";
+    case AR_EUNSUPPORTED: return "AR_EUNSUPPORTED: device is not sm_100 or size beyond limits";
+    case AR_ECUDA: return "AR_ECUDA: CUDA runtime call or kernel launch failed";
+    case AR_ETIMEDOUT: return "AR_ETIMEDOUT: bounded device wait expired";
+    default: return "unknown ar_status";
+    }
+}
+
+}  // extern "C"

@@ -94,7 +94,7 @@ def eps32(eps: float) -> float:
 
 
 def _draw(gen: torch.Generator, shape, mean: float, std: float, dtype: str) -> torch.Tensor:
-    x = torch.randn(shape, generator=gen, dtype=torch.float32)
+    x = torch.randn(shape, generator=gen, dtype=torch.float32, device=gen.device)
     if std != 1.0:
         x.mul_(std)
     if mean != 0.0:
@@ -125,14 +125,16 @@ class NormInputs:
 
 def make_norm_inputs(wl: NormWorkload, T: int, dtype: str | None = None, *, seed: int | None = None,
                      W: int | None = None, H: int | None = None,
-                     residual: bool | None = None) -> NormInputs:
+                     residual: bool | None = None, device: str = "cpu") -> NormInputs:
     """Inputs of one instance of a norm workload.  ``W``, ``H``, ``residual``
-    and ``seed`` may be overridden for edge-case tests (same distributions)."""
+    and ``seed`` may be overridden for edge-case tests (same distributions).
+    ``device="cuda"`` draws the same distributions with the device generator
+    (other values than the CPU draw; used only for timing)."""
     dtype = dtype or wl.dtypes[0]
     W = wl.W if W is None else W
     H = wl.H if H is None else H
     has_res = (wl.residual is not None) if residual is None else residual
-    gen = torch.Generator().manual_seed(seed_for(wl.name, T) if seed is None else seed)
+    gen = torch.Generator(device=device).manual_seed(seed_for(wl.name, T) if seed is None else seed)
     parts = [_draw(gen, (T, H), *wl.partial, dtype) for _ in range(W)]
     res = _draw(gen, (T, H), *(wl.residual or (0.0, 1.0)), dtype) if has_res else None
     wt = _draw(gen, (H,), *wl.weight, dtype)
@@ -155,12 +157,12 @@ class QKInputs:
 
 def make_qk_inputs(wl: QKWorkload, T: int, dtype: str | None = None, *, seed: int | None = None,
                    W: int | None = None, q_size: int | None = None,
-                   kv_size: int | None = None) -> QKInputs:
+                   kv_size: int | None = None, device: str = "cpu") -> QKInputs:
     dtype = dtype or wl.dtypes[0]
     W = wl.W if W is None else W
     q_size = wl.q_size if q_size is None else q_size
     kv_size = wl.kv_size if kv_size is None else kv_size
-    gen = torch.Generator().manual_seed(seed_for(wl.name, T) if seed is None else seed)
+    gen = torch.Generator(device=device).manual_seed(seed_for(wl.name, T) if seed is None else seed)
     row = q_size // W + 2 * (kv_size // W)
     shards = [_draw(gen, (T, row), *wl.act, dtype) for _ in range(W)]
     qw = _draw(gen, (q_size,), *wl.weight, dtype)

@@ -1,0 +1,200 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and
+loads, exports every entry point ``include/*.h`` declares, rejects bad
+arguments with the documented status before touching the device, treats
+T == 0 as a no-op, and loads / rejects plan tables as documented."""
+import ctypes
+import glob
+import json
+import os
+import re
+
+import pytest
+
+from tensor_allreduce_residual_ar_b200 import build as arbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, EINVAL, EALIGN, EUNSUP = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def clib():
+    path = arbuild.build()
+    lib = ctypes.CDLL(path)
+    P, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    lib.ar_add_rmsnorm.argtypes = [PP, P, P, P, P, i64, i64, i32, f32, i32, i32, P]
+    lib.ar_add_rmsnorm_quant_fp8_group.argtypes = [PP, P, P, P, P, P, P, i64, i64, i32, i32, f32,
+                                                   i32, i32, P]
+    lib.qk_norm_sharded.argtypes = [PP, P, P, PP, PP, i64, i64, i64, i32, f32, i32, P]
+    lib.ar_plan_query.argtypes = [i32, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_int)]
+    lib.ar_plan_load.argtypes = [ctypes.c_char_p]
+    lib.ar_plan_force.argtypes = [i32, i32]
+    lib.ar_status_string.restype = ctypes.c_char_p
+    yield lib
+    lib.ar_plan_load(None)
+    for v in range(3):
+        lib.ar_plan_force(v, 0)
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = "\n".join(l for l in open(h).read().splitlines() if not l.lstrip().startswith("#"))
+        names |= set(re.findall(r"AR_API\s+[\w\s\*]*?\b(\w+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(clib):
+    names = _declared_symbols()
+    assert {"ar_add_rmsnorm", "ar_add_rmsnorm_quant_fp8_group", "qk_norm_sharded",
+            "ar_plan_query", "ar_status_string"} <= names
+    for n in names:
+        assert hasattr(clib, n), n
+
+
+def test_library_has_no_oracle_dependency():
+    """The product library links nothing from the oracle."""
+    for src in arbuild.sources() + glob.glob(os.path.join(ROOT, "tensor_allreduce_residual_ar_b200", "*.py")):
+        text = open(src).read()
+        assert "oracle" not in re.sub(r"#.*|//.*", "", text).lower() or src.endswith("workloads.py"), src
+
+
+def _ptrs(*vals):
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+A = 0x100000          # fake, 16-byte aligned device addresses: never dereferenced
+B, C_, D, E = A + 0x1000, A + 0x2000, A + 0x3000, A + 0x4000
+
+
+def test_norm_argument_errors(clib):
+    parts = _ptrs(A, B)
+    f = clib.ar_add_rmsnorm
+    assert f(None, None, C_, D, None, 4, 64, 2, 1e-6, 0, 0, None) == EINVAL
+    assert f(parts, None, None, D, None, 4, 64, 2, 1e-6, 0, 0, None) == EINVAL      # weight
+    assert f(parts, None, C_, None, None, 4, 64, 2, 1e-6, 0, 0, None) == EINVAL     # out
+    assert f(parts, None, C_, D, None, 4, 60, 2, 1e-6, 0, 0, None) == EINVAL        # H % 8
+    assert f(parts, None, C_, D, None, 4, 0, 2, 1e-6, 0, 0, None) == EINVAL
+    assert f(parts, None, C_, D, None, -1, 64, 2, 1e-6, 0, 0, None) == EINVAL
+    assert f(parts, None, C_, D, None, 4, 64, 0, 1e-6, 0, 0, None) == EINVAL        # W
+    assert f(_ptrs(*([A] * 17)), None, C_, D, None, 4, 64, 17, 1e-6, 0, 0, None) == EINVAL
+    assert f(parts, None, C_, D, None, 4, 64, 2, 1e-6, 0, 2, None) == EINVAL        # dtype
+    assert f(parts, None, C_, D, None, 4, 64, 2, -1.0, 0, 0, None) == EINVAL        # eps
+    assert f(parts, None, C_, D, None, 4, 64, 2, float("nan"), 0, 0, None) == EINVAL
+    assert f(_ptrs(A, None), None, C_, D, None, 4, 64, 2, 1e-6, 0, 0, None) == EINVAL
+    assert f(_ptrs(A, B + 2), None, C_, D, None, 4, 64, 2, 1e-6, 0, 0, None) == EALIGN
+    assert f(parts, E + 8, C_, D, None, 4, 64, 2, 1e-6, 0, 0, None) == EALIGN       # residual
+    assert f(parts, None, C_ + 4, D, None, 4, 64, 2, 1e-6, 0, 0, None) == EALIGN    # weight
+    assert f(parts, None, C_, D + 2, None, 4, 64, 2, 1e-6, 0, 0, None) == EALIGN    # out
+    assert f(parts, None, C_, D, E + 6, 4, 64, 2, 1e-6, 0, 0, None) == EALIGN       # res out
+    assert f(parts, None, C_, D, None, 4, 65536 + 8, 2, 1e-6, 0, 0, None) == EUNSUP
+    # T == 0: valid, nothing launched (no device needed)
+    assert f(parts, E, C_, D, E, 0, 64, 2, 1e-6, 1, 1, None) == OK
+
+
+def test_fp8_argument_errors(clib):
+    parts = _ptrs(A, B)
+    f = clib.ar_add_rmsnorm_quant_fp8_group
+    args = lambda **kw: dict(dict(q=D, s=E, y=None, ro=None, T=4, H=256, W=2, g=128), **kw)
+    def call(**kw):
+        a = args(**kw)
+        return f(parts, None, C_, a["q"], a["s"], a["y"], a["ro"], a["T"], a["H"], a["W"], a["g"],
+                 1e-6, 0, 0, None)
+    assert call(q=None) == EINVAL
+    assert call(s=None) == EINVAL
+    assert call(g=64) == EINVAL
+    assert call(H=200) == EINVAL            # H not a multiple of the group
+    assert call(q=D + 8) == EALIGN
+    assert call(s=E + 2) == EALIGN
+    assert call(y=A + 4) == EALIGN
+    assert call(s=E + 4, T=0) == OK         # scales need only 4-byte alignment
+
+
+def test_qk_argument_errors(clib):
+    f = clib.qk_norm_sharded
+    qkv, qo, ko = _ptrs(A, B), _ptrs(C_, D), _ptrs(E, E + 0x1000)
+    base = dict(T=3, q=64, kv=32, W=2)
+    def call(qkv=qkv, qo=qo, ko=ko, **kw):
+        a = dict(base, **kw)
+        return f(qkv, A, B, qo, ko, a["T"], a["q"], a["kv"], a["W"], 1e-6, 0, None)
+    assert call(q=63) == EINVAL             # not a multiple of W
+    assert call(q=48, kv=16, W=4) == EINVAL   # kv/W = 4 not a multiple of 8
+    assert call(kv=0) == EINVAL
+    assert call(W=0) == EINVAL
+    assert call(qkv=_ptrs(A, None)) == EINVAL
+    assert call(qo=_ptrs(C_, D + 2)) == EALIGN
+    assert call(T=0) == OK
+
+
+def test_status_strings(clib):
+    for s in range(6):
+        assert clib.ar_status_string(s).decode().startswith("AR_")
+    assert b"unknown" in clib.ar_status_string(99)
+
+
+def test_plan_table_load_and_reject(clib, tmp_path):
+    q = ctypes.c_int(-1)
+    clib.ar_plan_load(None)
+    assert clib.ar_plan_table_size() == 0
+    assert clib.ar_plan_query(0, 8192, 4096, 8, 0, ctypes.byref(q)) == OK
+    builtin = q.value
+    good = {"entries": [{"variant": 0, "dtype": 0, "W": 8, "H": 4096, "t_lo": 1, "t_hi": 100000,
+                         "plan": 3}]}
+    p = tmp_path / "good.json"
+    p.write_text(json.dumps(good))
+    assert clib.ar_plan_load(str(p).encode()) == OK
+    assert clib.ar_plan_table_size() == 1
+    assert clib.ar_plan_query(0, 8192, 4096, 8, 0, ctypes.byref(q)) == OK and q.value == 3
+    # other shapes still take the built-in rule
+    assert clib.ar_plan_query(0, 8192, 4096, 8, 1, ctypes.byref(q)) == OK and q.value == builtin
+    # corrupt or invalid tables are rejected and the loaded one stays
+    bad_texts = [
+        "{not json",
+        json.dumps({"entries": [{"variant": 0, "dtype": 0, "W": 8, "H": 4096, "t_lo": 1,
+                                 "t_hi": 9, "plan": 11}]}),          # QK plan for norm
+        json.dumps({"entries": [{"variant": 0, "dtype": 0, "W": 8, "H": 4096, "t_lo": 9,
+                                 "t_hi": 1, "plan": 1}]}),           # empty range
+        json.dumps({"entries": [{"variant": 0, "dtype": 0, "W": 8, "H": 4096, "t_lo": 1,
+                                 "t_hi": 9, "plna": 1}]}),           # typo
+        json.dumps({"entries": [{"variant": 0, "dtype": 0, "W": 8, "H": 4096, "t_lo": 1,
+                                 "t_hi": 9, "plan": 1.5}]}),         # not an integer
+        json.dumps({"entries": []}) + " trailing",
+    ]
+    for i, text in enumerate(bad_texts):
+        bp = tmp_path / f"bad{i}.json"
+        bp.write_text(text)
+        assert clib.ar_plan_load(str(bp).encode()) == EINVAL, text
+        assert clib.ar_plan_table_size() == 1
+    assert clib.ar_plan_load(str(tmp_path / "missing.json").encode()) == EINVAL
+    assert clib.ar_plan_load(None) == OK and clib.ar_plan_table_size() == 0
+
+
+def test_plan_force(clib):
+    q = ctypes.c_int(-1)
+    assert clib.ar_plan_force(0, 11) == EINVAL      # QK plan for the norm variant
+    assert clib.ar_plan_force(2, 1) == EINVAL
+    assert clib.ar_plan_force(3, 1) == EINVAL
+    assert clib.ar_plan_force(1, 4) == OK
+    assert clib.ar_plan_query(1, 5, 5120, 4, 0, ctypes.byref(q)) == OK and q.value == 4
+    assert clib.ar_plan_force(1, 0) == OK
+    assert clib.ar_plan_query(2, 1, 7168, 8, 0, ctypes.byref(q)) == OK and 11 <= q.value <= 14
+
+
+def test_builtin_rule_is_capture_static(clib):
+    """Same arguments, same plan, however often asked (no state, no data)."""
+    q1, q2 = ctypes.c_int(-1), ctypes.c_int(-1)
+    clib.ar_plan_load(None)
+    for T in (1, 2, 80, 81, 4096, 8192, 32768):
+        for v, H in ((0, 8192), (1, 5120), (2, 7168)):
+            assert clib.ar_plan_query(v, T, H, 4 if v < 2 else 8, 0, ctypes.byref(q1)) == OK
+            assert clib.ar_plan_query(v, T, H, 4 if v < 2 else 8, 0, ctypes.byref(q2)) == OK
+            assert q1.value == q2.value
+
+
+def test_shipped_plan_table_parses(clib):
+    path = os.path.join(ROOT, "tensor_allreduce_residual_ar_b200", "plan_table.json")
+    if not os.path.exists(path):
+        pytest.skip("no plan table shipped yet")
+    assert clib.ar_plan_load(path.encode()) == OK
+    assert clib.ar_plan_table_size() > 0
+    clib.ar_plan_load(None)
