@@ -457,6 +457,27 @@ def run_reference(args):
     return 0
 
 
+def run_launches(args):
+    """Profiling mode: every call of the workload `--launches` times, plain
+    stream launches (no graph, no timing), for a profiler to capture."""
+    import torch
+    import tensor_allreduce_residual_ar_b200 as ar
+    device = torch.device("cuda", dist_env()[2])
+    torch.cuda.set_device(device)
+    ar.load_library()
+    calls = workload_calls(args.workload)
+    if args.only_T:
+        calls = [c for c in calls if c[2] in args.only_T]
+    bufs = [CallBuffers(c, device) for c in calls]
+    for _ in range(args.launches):
+        for b in bufs:
+            b.run(ar)
+    torch.cuda.synchronize()
+    print(json.dumps({"launches": args.launches * len(bufs), "workload": args.workload,
+                      "calls": [[c[2], c[3], plan_of(ar, c)] for c in calls]}))
+    return 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -489,7 +510,7 @@ def run_ours(args):
     # warm-up: W steps, then enough untimed steps to bring clocks to load
     time_graphs(graphs, max(3, args.warmup), stream)
     est = time_graphs(graphs, 20, stream) / 20
-    spin = int(min(20000, max(10, 0.5 / max(est, 1e-7))))   # ~0.5 s of load
+    spin = int(min(20000, max(10, args.spin_seconds / max(est, 1e-7))))   # load before timing
     sampler = ClockSampler(device.index)
     with sampler:
         time_graphs(graphs, spin, stream)
@@ -566,11 +587,19 @@ def main(argv=None):
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--spin-seconds", type=float, default=0.5,
+                    help="untimed load before the timed region (clocks settle, sampler runs)")
+    ap.add_argument("--launches", type=int, default=0,
+                    help="profiling mode: run every call this many times and exit")
+    ap.add_argument("--only-T", type=int, nargs="*", default=None,
+                    help="profiling mode: restrict to these T")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.launches:
+        return run_launches(args)
     return run_ours(args)
 
 

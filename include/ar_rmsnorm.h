@@ -177,10 +177,12 @@ AR_API int qk_norm_sharded(const void *const *qkv, const void *q_weight,
 typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_variant;
 
 /* Plan ids.  ROWC<k>: one row per cluster of k CTAs (sum of squares combined
- * through distributed shared memory).  PERSIST: one CTA per row, grid sized
- * to the SM count, rows looped.  BULK: PERSIST with rows staged into shared
- * memory by bulk asynchronous copies.  QK_C<k>: one token per cluster of k
- * CTAs, shards split across the cluster. */
+ * through distributed shared memory).  PERSIST / PERSIST512: one CTA of at
+ * most 256 / 512 threads per row, grid sized to the SM count x occupancy,
+ * rows looped, each CTA's next row bulk-prefetched into L2.  BULK: rows
+ * staged into shared memory by bulk asynchronous copies.  QK_C<k>: one token
+ * per cluster of k CTAs, shards split across the cluster; QK_PERSIST: one
+ * CTA per token, persistent grid with L2 prefetch. */
 enum {
     AR_PLAN_AUTO = 0,
     AR_PLAN_ROWC1 = 1,
@@ -189,10 +191,12 @@ enum {
     AR_PLAN_ROWC8 = 4,
     AR_PLAN_PERSIST = 5,
     AR_PLAN_BULK = 6,
+    AR_PLAN_PERSIST512 = 7,
     AR_PLAN_QK_C1 = 11,
     AR_PLAN_QK_C2 = 12,
     AR_PLAN_QK_C4 = 13,
-    AR_PLAN_QK_C8 = 14
+    AR_PLAN_QK_C8 = 14,
+    AR_PLAN_QK_PERSIST = 15
 };
 
 /* The plan a call with these arguments would use (for QK, H = q_size + kv_size

@@ -215,6 +215,7 @@ int run_norm(const void *const *partials, const void *residual, const void *weig
     }
     p.C = g.C;
     p.ppc = ppc;
+    p.prefetch = g.persistent ? 1 : 0;
     NormKernel fn = pick_norm_kernel(dtype, fp8, wb_bucket(W), ppt_idx);
     const int64_t clusters = grid_clusters(T, g, (const void *)fn, threads, dev, di.sm_count);
     return launch(fn, p, clusters, g.C, threads, stream);
@@ -307,8 +308,10 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
         // a token too wide for this plan's cluster: split it over more CTAs
         if (g.C >= 8 || W % (2 * g.C) != 0) return AR_EUNSUPPORTED;
         g.C *= 2;
+        g.persistent = false;
     }
     p.C = g.C;
+    p.prefetch = g.persistent ? 1 : 0;
     QKKernel fn = pick_qk_kernel(dtype, ppt_idx);
     const int64_t clusters = grid_clusters(T, g, (const void *)fn, threads, dev, di.sm_count);
     return launch(fn, p, clusters, g.C, threads, stream);

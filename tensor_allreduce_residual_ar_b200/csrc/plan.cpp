@@ -33,8 +33,10 @@ std::mutex g_load_mutex;
 std::vector<const Table *> g_retired;
 std::atomic<int> g_force[3] = {{0}, {0}, {0}};
 
-bool is_norm_plan(int id) { return id >= AR_PLAN_ROWC1 && id <= AR_PLAN_PERSIST; }
-bool is_qk_plan(int id) { return id >= AR_PLAN_QK_C1 && id <= AR_PLAN_QK_C8; }
+bool is_norm_plan(int id) {
+    return (id >= AR_PLAN_ROWC1 && id <= AR_PLAN_PERSIST) || id == AR_PLAN_PERSIST512;
+}
+bool is_qk_plan(int id) { return id >= AR_PLAN_QK_C1 && id <= AR_PLAN_QK_PERSIST; }
 
 // Minimal reader for {"entries": [{"key": int, ...}, ...]}: every value must
 // be an integer; unknown keys are errors, so a typo cannot silently drop a
@@ -152,10 +154,12 @@ Geometry plan_geometry(int id) {
     case AR_PLAN_ROWC4: return {4, false, 512};
     case AR_PLAN_ROWC8: return {8, false, 512};
     case AR_PLAN_PERSIST: return {1, true, 256};
+    case AR_PLAN_PERSIST512: return {1, true, 512};
     case AR_PLAN_QK_C1: return {1, false, 512};
     case AR_PLAN_QK_C2: return {2, false, 512};
     case AR_PLAN_QK_C4: return {4, false, 512};
     case AR_PLAN_QK_C8: return {8, false, 512};
+    case AR_PLAN_QK_PERSIST: return {1, true, 256};
     default: return {1, false, 512};
     }
 }

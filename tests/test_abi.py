@@ -198,3 +198,25 @@ def test_shipped_plan_table_parses(clib):
     assert clib.ar_plan_load(path.encode()) == OK
     assert clib.ar_plan_table_size() > 0
     clib.ar_plan_load(None)
+
+
+def test_tuner_ranges_cover_every_T(clib, tmp_path):
+    """The tuner's measured winners become contiguous T ranges that the
+    library accepts and that reproduce every winner."""
+    from tensor_allreduce_residual_ar_b200.tune import table_from_best
+    best = {(0, 0, 4, 8192, 1): 4, (0, 0, 4, 8192, 2): 4, (0, 0, 4, 8192, 16): 3,
+            (0, 0, 4, 8192, 80): 2, (1, 0, 4, 5120, 1): 4, (1, 0, 4, 5120, 4096): 5,
+            (2, 0, 8, 7168, 1): 14, (2, 0, 8, 7168, 2048): 15}
+    table = table_from_best(best)
+    assert len(table["entries"]) == 7          # the two T=1,2 plan-4 ranges merged
+    p = tmp_path / "t.json"
+    p.write_text(json.dumps(table))
+    assert clib.ar_plan_load(str(p).encode()) == OK
+    q = ctypes.c_int(-1)
+    for (v, d, W, H, T), plan in best.items():
+        assert clib.ar_plan_query(v, T, H, W, d, ctypes.byref(q)) == OK and q.value == plan
+    # between measured points the next measured point's plan applies; beyond
+    # the last one the last plan does
+    assert clib.ar_plan_query(0, 10, 8192, 4, 0, ctypes.byref(q)) == OK and q.value == 3
+    assert clib.ar_plan_query(0, 10**6, 8192, 4, 0, ctypes.byref(q)) == OK and q.value == 2
+    clib.ar_plan_load(None)
