@@ -217,6 +217,26 @@ AR_API int ar_plan_load(const char *path);
  * measurement; AR_EINVAL for an id that does not belong to the variant. */
 AR_API int ar_plan_force(int variant, int plan_id);
 
+/*
+ * Device-side status.  The bulk-staged kernel (AR_PLAN_BULK) bounds every
+ * wait on its copy pipeline; a wait that sees no progress for one second
+ * makes the kernel record AR_ETIMEDOUT here and wind down (its outputs for
+ * the affected rows are then undefined).  ar_device_status synchronises the
+ * current device, returns AR_ETIMEDOUT if any launch on it recorded a timeout
+ * since the last clear (AR_OK otherwise, AR_ECUDA if the device could not be
+ * read), and clears the record when `clear` is non-zero.
+ */
+AR_API int ar_device_status(int clear);
+
+/*
+ * Test hook for the bounded waits: the next bulk-staged launch on any device
+ * never issues the copies of row `row` (>= 0), so that row's consumers wait
+ * out their limit; -1 (the default) disables it.  The hook resets itself
+ * after one launch.  It exists so failure handling can be tested without a
+ * GPU fault; production code never sets it.
+ */
+AR_API int ar_test_withhold_row(int64_t row);
+
 /* Number of table entries currently loaded. */
 AR_API int ar_plan_table_size(void);
 

@@ -5,6 +5,7 @@ The compute lives in a C-ABI CUDA library (``csrc/``, header
 """
 from .binding import (  # noqa: F401
     AR_BF16, AR_FP16, ARError, ar_add_rmsnorm, ar_add_rmsnorm_quant_fp8_group,
-    ar_plan_force, ar_plan_load, ar_plan_query, ar_plan_table_size, ar_status_string,
+    ar_device_status, ar_plan_force, ar_plan_load, ar_plan_query, ar_plan_table_size,
+    ar_status_string, ar_test_withhold_row,
     library_path, load_library, qk_norm_sharded,
 )

@@ -66,6 +66,10 @@ def load_library():
         lib.ar_plan_table_size.argtypes = []
         lib.ar_status_string.restype = ctypes.c_char_p
         lib.ar_status_string.argtypes = [i32]
+        lib.ar_device_status.restype = i32
+        lib.ar_device_status.argtypes = [i32]
+        lib.ar_test_withhold_row.restype = i32
+        lib.ar_test_withhold_row.argtypes = [i64]
         if os.path.exists(_PLAN_TABLE):
             st = lib.ar_plan_load(_PLAN_TABLE.encode())
             if st != 0:
@@ -169,3 +173,14 @@ def ar_plan_force(variant: int, plan_id: int) -> int:
 
 def ar_plan_table_size() -> int:
     return load_library().ar_plan_table_size()
+
+
+def ar_device_status(clear: bool = True) -> int:
+    """Synchronise the current device; AR_ETIMEDOUT (5) if a bounded device
+    wait ran out since the last clear, else 0."""
+    return load_library().ar_device_status(int(bool(clear)))
+
+
+def ar_test_withhold_row(row: int) -> int:
+    """Test hook: the next bulk-staged launch never issues row `row`'s copies."""
+    return load_library().ar_test_withhold_row(int(row))

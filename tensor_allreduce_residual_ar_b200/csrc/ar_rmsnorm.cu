@@ -6,6 +6,7 @@
 // and no try/except-style fallback that hides a failure (PR #44849 report,
 // section 评论区精华).  Every rejection is a status code, and nothing is
 // launched after a rejection.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -22,6 +23,7 @@ constexpr int kMaxDevices = 64;
 
 struct DevInfo {
     int sm_count = 0;
+    int smem_optin = 0;   // largest dynamic shared memory per block
     int status = AR_OK;
 };
 
@@ -35,15 +37,17 @@ int device_info(DevInfo &out) {
     if (cudaGetDevice(&dev) != cudaSuccess) return AR_ECUDA;
     if (dev < 0 || dev >= kMaxDevices) return AR_EUNSUPPORTED;
     std::call_once(g_dev_once[dev], [dev] {
-        int major = 0, minor = 0, sms = 0;
+        int major = 0, minor = 0, sms = 0, optin = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
             g_dev[dev].status = AR_ECUDA;
             return;
         }
         g_dev[dev].status = (major == 10 && minor == 0) ? AR_OK : AR_EUNSUPPORTED;
         g_dev[dev].sm_count = sms;
+        g_dev[dev].smem_optin = optin;
     });
     out = g_dev[dev];
     return out.status;
@@ -62,9 +66,9 @@ int wb_bucket(int W) { return W <= 2 ? 0 : W <= 4 ? 1 : W <= 8 ? 2 : 3; }   // 2
 using NormKernel = void (*)(const NormParams);
 using QKKernel = void (*)(const QKParams);
 
-template <typename Elt, bool FP8>
+template <typename Elt, bool FP8, int MINB>
 NormKernel norm_kernel_for(int wb, int ppt_idx) {
-#define ARN_K(WB, PPT) &norm_rows_kernel<Elt, WB, PPT, FP8>
+#define ARN_K(WB, PPT) &norm_rows_kernel<Elt, WB, PPT, FP8, MINB>
     static const NormKernel tab[4][kPptVariants] = {
         {ARN_K(2, 1), ARN_K(2, 2), ARN_K(2, 4)},
         {ARN_K(4, 1), ARN_K(4, 2), ARN_K(4, 4)},
@@ -75,20 +79,76 @@ NormKernel norm_kernel_for(int wb, int ppt_idx) {
     return tab[wb][ppt_idx];
 }
 
-NormKernel pick_norm_kernel(int dtype, bool fp8, int wb, int ppt_idx) {
+NormKernel pick_norm_kernel(int dtype, bool fp8, int wb, int ppt_idx, int minb) {
+    if (minb == 2) {
+        if (dtype == AR_BF16)
+            return fp8 ? norm_kernel_for<__nv_bfloat16, true, 2>(wb, ppt_idx)
+                       : norm_kernel_for<__nv_bfloat16, false, 2>(wb, ppt_idx);
+        return fp8 ? norm_kernel_for<__half, true, 2>(wb, ppt_idx) : norm_kernel_for<__half, false, 2>(wb, ppt_idx);
+    }
     if (dtype == AR_BF16)
-        return fp8 ? norm_kernel_for<__nv_bfloat16, true>(wb, ppt_idx)
-                   : norm_kernel_for<__nv_bfloat16, false>(wb, ppt_idx);
-    return fp8 ? norm_kernel_for<__half, true>(wb, ppt_idx) : norm_kernel_for<__half, false>(wb, ppt_idx);
+        return fp8 ? norm_kernel_for<__nv_bfloat16, true, 1>(wb, ppt_idx)
+                   : norm_kernel_for<__nv_bfloat16, false, 1>(wb, ppt_idx);
+    return fp8 ? norm_kernel_for<__half, true, 1>(wb, ppt_idx) : norm_kernel_for<__half, false, 1>(wb, ppt_idx);
 }
 
-QKKernel pick_qk_kernel(int dtype, int ppt_idx) {
-    static const QKKernel bf[kPptVariants] = {&qk_norm_kernel<__nv_bfloat16, 1>,
-                                              &qk_norm_kernel<__nv_bfloat16, 2>,
-                                              &qk_norm_kernel<__nv_bfloat16, 4>};
-    static const QKKernel hf[kPptVariants] = {&qk_norm_kernel<__half, 1>, &qk_norm_kernel<__half, 2>,
-                                              &qk_norm_kernel<__half, 4>};
-    return dtype == AR_BF16 ? bf[ppt_idx] : hf[ppt_idx];
+// Bulk-staged kernels: one slot of EPT elements per consumer thread.
+// EPT 4 with up to 1024 consumers (rows up to 4096 elements), EPT 8 with up
+// to 640 consumers (rows up to 5120 elements).
+constexpr int kBulkMaxT4 = 1024;
+constexpr int kBulkMaxT8 = 640;
+
+template <typename Elt, bool FP8>
+NormKernel bulk_kernel_for(int wb, int ept) {
+#define ARN_B(WB) ept == 4 ? &norm_bulk_kernel<Elt, WB, 4, FP8, kBulkMaxT4> \
+                           : &norm_bulk_kernel<Elt, WB, 8, FP8, kBulkMaxT8>
+    switch (wb) {
+    case 0: return ARN_B(2);
+    case 1: return ARN_B(4);
+    case 2: return ARN_B(8);
+    default: return ARN_B(16);
+    }
+#undef ARN_B
+}
+
+NormKernel pick_bulk_kernel(int dtype, bool fp8, int wb, int ept) {
+    if (dtype == AR_BF16)
+        return fp8 ? bulk_kernel_for<__nv_bfloat16, true>(wb, ept)
+                   : bulk_kernel_for<__nv_bfloat16, false>(wb, ept);
+    return fp8 ? bulk_kernel_for<__half, true>(wb, ept) : bulk_kernel_for<__half, false>(wb, ept);
+}
+
+// Opt a kernel into `bytes` of dynamic shared memory (once per kernel and
+// size class; kernel attributes are per device context, so the first call on
+// every device sets them).
+std::mutex g_attr_mutex;
+struct AttrSlot { const void *fn; int dev; int bytes; };
+AttrSlot g_attr[512];
+int g_attr_n = 0;
+
+int ensure_smem(const void *fn, int dev, int bytes) {
+    std::lock_guard<std::mutex> lk(g_attr_mutex);
+    for (int i = 0; i < g_attr_n; ++i)
+        if (g_attr[i].fn == fn && g_attr[i].dev == dev && g_attr[i].bytes >= bytes) return AR_OK;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return AR_ECUDA;
+    if (g_attr_n < 512) g_attr[g_attr_n++] = {fn, dev, bytes};
+    return AR_OK;
+}
+
+std::atomic<int64_t> g_withhold_row{-1};
+
+QKKernel pick_qk_kernel(int dtype, int ppt_idx, int minb) {
+    static const QKKernel bf[2][kPptVariants] = {
+        {&qk_norm_kernel<__nv_bfloat16, 1, 1>, &qk_norm_kernel<__nv_bfloat16, 2, 1>,
+         &qk_norm_kernel<__nv_bfloat16, 4, 1>},
+        {&qk_norm_kernel<__nv_bfloat16, 1, 2>, &qk_norm_kernel<__nv_bfloat16, 2, 2>,
+         &qk_norm_kernel<__nv_bfloat16, 4, 2>}};
+    static const QKKernel hf[2][kPptVariants] = {
+        {&qk_norm_kernel<__half, 1, 1>, &qk_norm_kernel<__half, 2, 1>, &qk_norm_kernel<__half, 4, 1>},
+        {&qk_norm_kernel<__half, 1, 2>, &qk_norm_kernel<__half, 2, 2>, &qk_norm_kernel<__half, 4, 2>}};
+    const int m = minb == 2 ? 1 : 0;
+    return dtype == AR_BF16 ? bf[m][ppt_idx] : hf[m][ppt_idx];
 }
 
 // Threads per CTA and packs per thread for `packs` packs per CTA: the
@@ -127,11 +187,11 @@ int occupancy(const void *fn, int threads, int dev) {
 
 template <typename Params>
 int launch(void (*fn)(const Params), const Params &p, int64_t clusters, int C, int threads,
-           cudaStream_t stream) {
+           cudaStream_t stream, size_t smem = 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(clusters * C), 1, 1);
     cfg.blockDim = dim3((unsigned)threads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     if (C > 1) {
@@ -196,8 +256,46 @@ int run_norm(const void *const *partials, const void *residual, const void *weig
     p.eps = (double)eps;
     p.gemma = gemma ? 1 : 0;
 
+    p.withhold_row = -1;
+    // certified fast sum for outputs with p significand bits (bf16 8,
+    // fp16 11): accept s when |s| >= u (2^(p+2) + 1) sum_k |s_k|, with a 1%
+    // margin for the (1 + O(Wu)) factors and the fp32 evaluation of the test
+    {
+        const int pbits = dtype == AR_BF16 ? 8 : 11;
+        p.kcert = (float)(std::ldexp(1.0, -24) * (std::ldexp(1.0, pbits + 2) + 1.0) * 1.01);
+    }
     const int variant = fp8 ? AR_VARIANT_FP8 : AR_VARIANT_NORM;
-    const int plan = plan_lookup(variant, T, H, W, dtype, di.sm_count);
+    int plan = plan_lookup(variant, T, H, W, dtype, di.sm_count);
+
+    if (plan == AR_PLAN_BULK) {
+        // one row of every stream per stage, at least two stages in shared
+        // memory, one slot of 4 (or else 8) elements per consumer thread;
+        // otherwise the persistent register-resident plan
+        const int NS = W + (residual ? 1 : 0);
+        const size_t stage_bytes = (size_t)NS * (size_t)H * 2;
+        const size_t budget = (size_t)di.smem_optin > 4096 ? (size_t)di.smem_optin - 4096 : 0;
+        int stages = (int)(budget / stage_bytes);
+        if (stages > kBulkMaxStages) stages = kBulkMaxStages;
+        int ept = 0;
+        if ((H / 8 + 31) / 32 * 32 <= kBulkMaxT8) ept = 8;
+        else if ((H / 4 + 31) / 32 * 32 <= kBulkMaxT4) ept = 4;
+        if (stages >= 2 && ept != 0) {
+            const int consumers = (int)(((H / ept) + 31) / 32 * 32);
+            p.C = 1;
+            p.ppc = p.P;
+            p.prefetch = 0;
+            p.stages = stages;
+            p.consumers = consumers;
+            p.withhold_row = g_withhold_row.exchange(-1);
+            NormKernel fn = pick_bulk_kernel(dtype, fp8, wb_bucket(W), ept);
+            const int smem = (int)(stages * stage_bytes);
+            int st2 = ensure_smem((const void *)fn, dev, smem);
+            if (st2 != AR_OK) return st2;
+            const int64_t grid = T < di.sm_count ? T : di.sm_count;
+            return launch(fn, p, grid, 1, consumers, stream, (size_t)smem);
+        }
+        plan = AR_PLAN_PERSIST;
+    }
     Geometry g = plan_geometry(plan);
     // never split a row into slices narrower than one FP8 group
     while (g.C > 1 && (p.P + g.C - 1) / g.C < kGroupPacks) g.C /= 2;
@@ -216,7 +314,7 @@ int run_norm(const void *const *partials, const void *residual, const void *weig
     p.C = g.C;
     p.ppc = ppc;
     p.prefetch = g.persistent ? 1 : 0;
-    NormKernel fn = pick_norm_kernel(dtype, fp8, wb_bucket(W), ppt_idx);
+    NormKernel fn = pick_norm_kernel(dtype, fp8, wb_bucket(W), ppt_idx, g.minb);
     const int64_t clusters = grid_clusters(T, g, (const void *)fn, threads, dev, di.sm_count);
     return launch(fn, p, clusters, g.C, threads, stream);
 }
@@ -312,7 +410,7 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
     }
     p.C = g.C;
     p.prefetch = g.persistent ? 1 : 0;
-    QKKernel fn = pick_qk_kernel(dtype, ppt_idx);
+    QKKernel fn = pick_qk_kernel(dtype, ppt_idx, g.minb);
     const int64_t clusters = grid_clusters(T, g, (const void *)fn, threads, dev, di.sm_count);
     return launch(fn, p, clusters, g.C, threads, stream);
 }
@@ -329,6 +427,23 @@ int ar_plan_query(int variant, int64_t T, int64_t H, int W, int dtype, int *plan
 }
 
 int ar_plan_load(const char *path) { return plan_load_file(path); }
+
+int ar_device_status(int clear) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return AR_ECUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, arn::g_ar_device_status, sizeof v) != cudaSuccess) return AR_ECUDA;
+    if (clear && v) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(arn::g_ar_device_status, &zero, sizeof zero) != cudaSuccess) return AR_ECUDA;
+    }
+    return v ? AR_ETIMEDOUT : AR_OK;
+}
+
+int ar_test_withhold_row(int64_t row) {
+    if (row < -1) return AR_EINVAL;
+    g_withhold_row.store(row);
+    return AR_OK;
+}
 
 int ar_plan_force(int variant, int plan_id) { return plan_force(variant, plan_id); }
 

@@ -17,6 +17,7 @@ struct Geometry {
     int C;            // CTAs per row / token (cluster size)
     bool persistent;  // grid capped at SM count x occupancy, rows looped
     int max_threads;  // upper bound on threads per CTA
+    int minb;         // CTAs per SM the kernel's registers are sized for (1 or 2)
 };
 
 bool plan_valid_for(int variant, int plan_id);

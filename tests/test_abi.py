@@ -126,6 +126,12 @@ def test_qk_argument_errors(clib):
     assert call(T=0) == OK
 
 
+def test_withhold_hook_validates(clib):
+    clib.ar_test_withhold_row.argtypes = [ctypes.c_int64]
+    assert clib.ar_test_withhold_row(-2) == EINVAL
+    assert clib.ar_test_withhold_row(-1) == OK
+
+
 def test_status_strings(clib):
     for s in range(6):
         assert clib.ar_status_string(s).decode().startswith("AR_")

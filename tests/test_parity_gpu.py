@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 
 GUARD = 512
 SENT16 = 0x5A5A
-NORM_PLANS = (1, 2, 3, 4, 5, 7)
+NORM_PLANS = (1, 2, 3, 4, 5, 6, 7)
 QK_PLANS = (11, 12, 13, 14, 15)
 TD = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -307,3 +307,42 @@ def test_three_d_tokens_flatten(lib):
     o = P.oracle_norm(inp)
     P.check_y(P.to_bits(out.view(12, 1024)), o["y"], "bf16")
     P.check_res(P.to_bits(rout.view(12, 1024)), o["r"], "bf16")
+
+
+def test_bulk_plan_wait_timeout_is_reported(lib):
+    """A bulk-staged launch whose row never lands: its consumers' bounded
+    wait runs out, the device status says AR_ETIMEDOUT, the context stays
+    usable, and the next call is correct with a clean status."""
+    inp = wl.make_norm_inputs(wl.PREFILL, 64, seed=41)
+    assert lib.ar_device_status(True) == 0
+    assert lib.ar_test_withhold_row(5) == 0
+    run_norm(lib, inp, plan=6)                 # finishes after the 1 s limit
+    assert lib.ar_device_status(True) == 5     # AR_ETIMEDOUT, now cleared
+    assert lib.ar_device_status(True) == 0
+    check_norm(lib, inp, plan=6)
+    assert lib.ar_device_status(True) == 0
+
+
+def test_bulk_plan_falls_back_when_rows_do_not_fit(lib):
+    """W=16, H=8192: 17 rows of 16 KiB per stage do not fit twice in shared
+    memory, so the bulk plan runs the persistent kernel instead."""
+    inp = wl.make_norm_inputs(wl.DECODE, 9, "bf16", W=16, H=8192, seed=42)
+    check_norm(lib, inp, plan=6)
+
+
+@pytest.mark.parametrize("plan", (1, 5, 6))
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_cancellation_sweep_around_certificate(lib, plan, dtype):
+    """residual = -(sum of partials) + delta * noise, rounded: r is small
+    against the terms at every scale delta, so elements land on both sides
+    of the fast-sum acceptance test and many take the exact fallback."""
+    T, H, W = 16, 2048, 6
+    gen = torch.Generator().manual_seed(7000 + plan)
+    td = TD[dtype]
+    parts = [torch.randn(T, H, generator=gen).to(td) for _ in range(W)]
+    total = sum(p.double() for p in parts)
+    scales = torch.tensor([1e-1, 1e-2, 1e-3, 1e-4, 1e-5, 0.0]).repeat_interleave(H // 6 + 1)[:H]
+    res = (-total + scales.double() * torch.randn(T, H, generator=gen).double()).to(td)
+    w = (1.0 + 0.1 * torch.randn(H, generator=gen)).to(td)
+    inp = wl.NormInputs(parts, res, w, T, H, W, dtype, wl.eps32(1e-6), False, True)
+    check_norm(lib, inp, plan=plan)
