@@ -300,17 +300,23 @@ def capture_step_graphs(ar, sets, stream):
     return graphs
 
 
-def time_graphs(graphs, n, stream):
+def time_graphs(graphs, n, stream, label=None):
+    """Replay n steps; the timed region carries an NVTX range `label` so a
+    profiler can restrict itself to it."""
     import torch
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    if label:
+        torch.cuda.nvtx.range_push(label)
     with torch.cuda.stream(stream):
         start.record(stream)
         for i in range(n):
             graphs[i % len(graphs)].replay()
         end.record(stream)
     end.synchronize()
+    if label:
+        torch.cuda.nvtx.range_pop()
     return start.elapsed_time(end) / 1e3
 
 
@@ -516,7 +522,7 @@ def run_ours(args):
         time_graphs(graphs, spin, stream)
         barrier(device)
         torch.cuda.synchronize()
-        el = time_graphs(graphs, args.steps, stream)
+        el = time_graphs(graphs, args.steps, stream, label="bench_timed")
         torch.cuda.synchronize()
         barrier(device)
     el_max = max_over_ranks(el, device)

@@ -46,10 +46,15 @@
  *     errors on `stream`, as for any kernel.
  *   - 16-bit formats: AR_BF16 (bfloat16) or AR_FP16 (IEEE half); all 16-bit
  *     tensors of one call share `dtype`.
- *   - Accumulation is fp32 with a compensated (error-free transformation)
- *     sum of the W+1 terms, so r is within one fp32 ulp of the exact sum;
- *     the sum of squares is combined across threads in fp64; outputs are
- *     rounded to nearest even.
+ *   - Arithmetic is fp32.  The W+1 terms are summed with a certificate:
+ *     a plain fp32 sum is kept when its rounding-error bound is below
+ *     2^-(p+2) of the result (p = 8 for bf16, 11 for fp16 outputs), and
+ *     otherwise the element is recomputed with an error-free (TwoSum)
+ *     compensated sum; the FP8 variant always uses the compensated sum.
+ *     residual_out is therefore within one unit in the last place of the
+ *     rounded exact sum.  The sum of squares is combined across threads in
+ *     fp64 for the FP8 variant (its scales must be within 1e-6) and in fp32
+ *     otherwise.  Outputs are rounded to nearest even.
  */
 #ifndef AR_RMSNORM_H
 #define AR_RMSNORM_H

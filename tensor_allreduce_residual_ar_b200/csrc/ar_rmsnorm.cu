@@ -8,6 +8,7 @@
 // launched after a rejection.
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <mutex>
 
@@ -185,6 +186,16 @@ int occupancy(const void *fn, int threads, int dev) {
     return occ;
 }
 
+// Programmatic dependent launch is on unless AR_RMSNORM_PDL=0 in the
+// environment when the library first launches.
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("AR_RMSNORM_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
 template <typename Params>
 int launch(void (*fn)(const Params), const Params &p, int64_t clusters, int C, int threads,
            cudaStream_t stream, size_t smem = 0) {
@@ -193,15 +204,24 @@ int launch(void (*fn)(const Params), const Params &p, int64_t clusters, int C, i
     cfg.blockDim = dim3((unsigned)threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    int na = 0;
     if (C > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)C;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)C;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
     }
+    if (pdl_enabled()) {
+        // may start while the previous kernel in the stream finishes; the
+        // kernel waits for it (griddepcontrol.wait) before any memory access
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, fn, p) == cudaSuccess ? AR_OK : AR_ECUDA;
 }
 
