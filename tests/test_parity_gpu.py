@@ -346,3 +346,23 @@ def test_cancellation_sweep_around_certificate(lib, plan, dtype):
     w = (1.0 + 0.1 * torch.randn(H, generator=gen)).to(td)
     inp = wl.NormInputs(parts, res, w, T, H, W, dtype, wl.eps32(1e-6), False, True)
     check_norm(lib, inp, plan=plan)
+
+
+@pytest.mark.parametrize("plan", NORM_PLANS)
+def test_fp8_rare_accuracy_paths(lib, plan):
+    """Crafted rows that drive the FP8 variant's rare paths:
+    row 0, group 0: the group maximum has a large partial-sum bound
+    (100 - 50 - 45 + 5 = 10, bound 65 > 4 * 10), so it is recomputed exactly
+    before the scale is formed; row 1: residual ~ -(sum of partials), so the
+    sum-of-squares error bound is large and the whole row is recomputed;
+    rows 2-3 ordinary."""
+    T, H, W = 4, 256, 3
+    gen = torch.Generator().manual_seed(4242 + plan)
+    parts = [(0.5 * torch.randn(T, H, generator=gen)).to(torch.bfloat16) for _ in range(W)]
+    res = torch.randn(T, H, generator=gen).to(torch.bfloat16)
+    res[0, 0], parts[0][0, 0], parts[1][0, 0], parts[2][0, 0] = 100.0, -50.0, -45.0, 5.0
+    total = sum(p[1].double() for p in parts)
+    res[1] = (-total + 1e-3 * torch.randn(H, generator=gen).double()).to(torch.bfloat16)
+    w = (1.0 + 0.1 * torch.randn(H, generator=gen)).to(torch.bfloat16)
+    inp = wl.NormInputs(parts, res, w, T, H, W, "bf16", wl.eps32(1e-6), False, True)
+    check_fp8(lib, inp, plan=plan)
