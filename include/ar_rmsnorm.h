@@ -184,7 +184,9 @@ typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_v
 /* Plan ids.  ROWC<k>: one row per cluster of k CTAs (sum of squares combined
  * through distributed shared memory).  PERSIST / PERSIST512: one CTA of at
  * most 256 / 512 threads per row, grid sized to the SM count x occupancy,
- * rows looped, each CTA's next row bulk-prefetched into L2.  BULK: rows
+ * rows looped, each CTA's next row bulk-prefetched into L2.  PERSIST_C2: the
+ * same with each row split over a cluster of 2 CTAs (at most 512 threads
+ * each), the grid sized to the clusters that fit at once.  BULK: rows
  * staged into shared memory by bulk asynchronous copies.  QK_C<k>: one token
  * per cluster of k CTAs, shards split across the cluster; QK_PERSIST: one
  * CTA per token, persistent grid with L2 prefetch. */
@@ -197,6 +199,7 @@ enum {
     AR_PLAN_PERSIST = 5,
     AR_PLAN_BULK = 6,
     AR_PLAN_PERSIST512 = 7,
+    AR_PLAN_PERSIST_C2 = 8,
     AR_PLAN_QK_C1 = 11,
     AR_PLAN_QK_C2 = 12,
     AR_PLAN_QK_C4 = 13,

@@ -225,11 +225,48 @@ int launch(void (*fn)(const Params), const Params &p, int64_t clusters, int C, i
     return cudaLaunchKernelEx(&cfg, fn, p) == cudaSuccess ? AR_OK : AR_ECUDA;
 }
 
+// Clusters of C CTAs of a kernel that can be resident at once on the whole
+// device (cluster placement within GPCs included), cached.
+struct ClusterOccSlot { OccKey key; int C; int n; };
+ClusterOccSlot g_cocc[64];
+int g_cocc_n = 0;
+
+int cluster_occupancy(const void *fn, int threads, int C, int dev, int sm_count) {
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mutex);
+        for (int i = 0; i < g_cocc_n; ++i)
+            if (g_cocc[i].key.fn == fn && g_cocc[i].key.threads == threads &&
+                g_cocc[i].key.dev == dev && g_cocc[i].C == C)
+                return g_cocc[i].n;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)C, 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)C;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        n = sm_count * occupancy(fn, threads, dev) / C;
+    }
+    if (n < 1) n = 1;
+    std::lock_guard<std::mutex> lk(g_occ_mutex);
+    if (g_cocc_n < 64) g_cocc[g_cocc_n++] = {{fn, threads, dev}, C, n};
+    return n;
+}
+
 // Grid size in clusters: one per row, or capped for persistent plans.
 int64_t grid_clusters(int64_t rows, const Geometry &g, const void *fn, int threads, int dev,
                       int sm_count) {
     int64_t cap = (int64_t)0x7FFFFFFF / g.C;
-    if (g.persistent) cap = (int64_t)sm_count * occupancy(fn, threads, dev) / g.C;
+    if (g.persistent)
+        cap = g.C > 1 ? (int64_t)cluster_occupancy(fn, threads, g.C, dev, sm_count)
+                      : (int64_t)sm_count * occupancy(fn, threads, dev);
     if (cap < 1) cap = 1;
     return rows < cap ? rows : cap;
 }
