@@ -67,9 +67,9 @@ int wb_bucket(int W) { return W <= 2 ? 0 : W <= 4 ? 1 : W <= 8 ? 2 : 3; }   // 2
 using NormKernel = void (*)(const NormParams);
 using QKKernel = void (*)(const QKParams);
 
-template <typename Elt, bool FP8, int MINB>
+template <typename Elt, bool FP8, int MODE>
 NormKernel norm_kernel_for(int wb, int ppt_idx) {
-#define ARN_K(WB, PPT) &norm_rows_kernel<Elt, WB, PPT, FP8, MINB>
+#define ARN_K(WB, PPT) &norm_rows_kernel<Elt, WB, PPT, FP8, MODE>
     static const NormKernel tab[4][kPptVariants] = {
         {ARN_K(2, 1), ARN_K(2, 2), ARN_K(2, 4)},
         {ARN_K(4, 1), ARN_K(4, 2), ARN_K(4, 4)},
@@ -80,17 +80,20 @@ NormKernel norm_kernel_for(int wb, int ppt_idx) {
     return tab[wb][ppt_idx];
 }
 
-NormKernel pick_norm_kernel(int dtype, bool fp8, int wb, int ppt_idx, int minb) {
-    if (minb == 2) {
-        if (dtype == AR_BF16)
-            return fp8 ? norm_kernel_for<__nv_bfloat16, true, 2>(wb, ppt_idx)
-                       : norm_kernel_for<__nv_bfloat16, false, 2>(wb, ppt_idx);
-        return fp8 ? norm_kernel_for<__half, true, 2>(wb, ppt_idx) : norm_kernel_for<__half, false, 2>(wb, ppt_idx);
-    }
+template <int MODE>
+NormKernel pick_norm_kernel_mode(int dtype, bool fp8, int wb, int ppt_idx) {
     if (dtype == AR_BF16)
-        return fp8 ? norm_kernel_for<__nv_bfloat16, true, 1>(wb, ppt_idx)
-                   : norm_kernel_for<__nv_bfloat16, false, 1>(wb, ppt_idx);
-    return fp8 ? norm_kernel_for<__half, true, 1>(wb, ppt_idx) : norm_kernel_for<__half, false, 1>(wb, ppt_idx);
+        return fp8 ? norm_kernel_for<__nv_bfloat16, true, MODE>(wb, ppt_idx)
+                   : norm_kernel_for<__nv_bfloat16, false, MODE>(wb, ppt_idx);
+    return fp8 ? norm_kernel_for<__half, true, MODE>(wb, ppt_idx)
+               : norm_kernel_for<__half, false, MODE>(wb, ppt_idx);
+}
+
+// The kernel compiled for a plan's grid shape (see kModeRow and friends).
+NormKernel pick_norm_kernel(int dtype, bool fp8, int wb, int ppt_idx, const Geometry &g) {
+    if (g.minb == 2) return pick_norm_kernel_mode<kModePersist512>(dtype, fp8, wb, ppt_idx);
+    if (g.persistent) return pick_norm_kernel_mode<kModePersist>(dtype, fp8, wb, ppt_idx);
+    return pick_norm_kernel_mode<kModeRow>(dtype, fp8, wb, ppt_idx);
 }
 
 // Bulk-staged kernels: one slot of EPT elements per consumer thread.
@@ -371,7 +374,7 @@ int run_norm(const void *const *partials, const void *residual, const void *weig
     p.C = g.C;
     p.ppc = ppc;
     p.prefetch = g.persistent ? 1 : 0;
-    NormKernel fn = pick_norm_kernel(dtype, fp8, wb_bucket(W), ppt_idx, g.minb);
+    NormKernel fn = pick_norm_kernel(dtype, fp8, wb_bucket(W), ppt_idx, g);
     const int64_t clusters = grid_clusters(T, g, (const void *)fn, threads, dev, di.sm_count);
     return launch(fn, p, clusters, g.C, threads, stream);
 }
