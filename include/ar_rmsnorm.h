@@ -50,7 +50,9 @@
  *     a plain fp32 sum is kept when its rounding-error bound is below
  *     2^-(p+2) of the result (p = 8 for bf16, 11 for fp16 outputs), and
  *     otherwise the element is recomputed with an error-free (TwoSum)
- *     compensated sum; the FP8 variant always uses the compensated sum.
+ *     compensated sum.  The FP8 variant sums exactly: the fp32 sum rounded
+ *     down and rounded up agree exactly when it is exact, and elements where
+ *     they differ take the compensated sum.
  *     residual_out is therefore within one unit in the last place of the
  *     rounded exact sum.  The sum of squares is combined across threads in
  *     fp64 for the FP8 variant (its scales must be within 1e-6) and in fp32
