@@ -191,7 +191,8 @@ typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_v
  * each), the grid sized to the clusters that fit at once.  BULK: rows
  * staged into shared memory by bulk asynchronous copies.  QK_C<k>: one token
  * per cluster of k CTAs, shards split across the cluster; QK_PERSIST: one
- * CTA per token, persistent grid with L2 prefetch. */
+ * CTA (at most 512 threads) per token, persistent grid with L2 prefetch;
+ * QK_PERSIST256: the same with at most 256 threads (more packs per thread). */
 enum {
     AR_PLAN_AUTO = 0,
     AR_PLAN_ROWC1 = 1,
@@ -206,7 +207,8 @@ enum {
     AR_PLAN_QK_C2 = 12,
     AR_PLAN_QK_C4 = 13,
     AR_PLAN_QK_C8 = 14,
-    AR_PLAN_QK_PERSIST = 15
+    AR_PLAN_QK_PERSIST = 15,
+    AR_PLAN_QK_PERSIST256 = 16
 };
 
 /* The plan a call with these arguments would use (for QK, H = q_size + kv_size

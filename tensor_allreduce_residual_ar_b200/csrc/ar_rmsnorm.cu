@@ -449,9 +449,9 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
     p.qsp = (int)(qs / 8);
     p.ksp = (int)(ks / 8);
     p.row_packs = p.qsp + 2 * p.ksp;
-    p.inv_q = 1.0 / (double)q_size;
-    p.inv_k = 1.0 / (double)kv_size;
-    p.eps = (double)eps;
+    p.inv_q = (float)(1.0 / (double)q_size);
+    p.inv_k = (float)(1.0 / (double)kv_size);
+    p.eps = eps;
 
     const int plan = plan_lookup(AR_VARIANT_QK, T, q_size + kv_size, W, dtype, di.sm_count);
     Geometry g = plan_geometry(plan);

@@ -183,6 +183,10 @@ def test_plan_force(clib):
     assert clib.ar_plan_force(0, 8) == OK           # PERSIST_C2, the last norm plan
     assert clib.ar_plan_force(0, 9) == EINVAL
     assert clib.ar_plan_force(2, 8) == EINVAL
+    assert clib.ar_plan_force(2, 16) == OK          # QK_PERSIST256, the last QK plan
+    assert clib.ar_plan_force(2, 17) == EINVAL
+    assert clib.ar_plan_force(0, 16) == EINVAL
+    assert clib.ar_plan_force(2, 0) == OK
     assert clib.ar_plan_force(0, 0) == OK
     assert clib.ar_plan_force(1, 4) == OK
     assert clib.ar_plan_query(1, 5, 5120, 4, 0, ctypes.byref(q)) == OK and q.value == 4

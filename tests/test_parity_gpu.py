@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 GUARD = 512
 SENT16 = 0x5A5A
 NORM_PLANS = (1, 2, 3, 4, 5, 6, 7, 8)
-QK_PLANS = (11, 12, 13, 14, 15)
+QK_PLANS = (11, 12, 13, 14, 15, 16)
 TD = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
 
@@ -201,6 +201,17 @@ def test_norm_every_plan_ragged(lib, plan, T, H, W):
         check_norm(lib, inp, plan=plan, residual=res)
 
 
+def test_persistent_cluster_many_rows_per_cluster(lib):
+    """Plan PERSIST_C2 on shapes where every 2-CTA cluster reduces about
+    seven rows: the row partials' buffers and their barriers' phases are
+    reused many times (fp32 partials for 16-bit outputs, fp64 for FP8)."""
+    for dtype in ("bf16", "fp16"):
+        inp = wl.make_norm_inputs(wl.DECODE, 1000, dtype, W=4, H=8192, seed=808)
+        check_norm(lib, inp, plan=8)
+    inp = wl.make_norm_inputs(wl.FP8, 1500, W=4, H=5120, seed=809)
+    check_fp8(lib, inp, plan=8)
+
+
 @pytest.mark.parametrize("plan", NORM_PLANS)
 def test_norm_max_hidden(lib, plan):
     inp = wl.make_norm_inputs(wl.TINY, 3, W=2, H=65536, seed=65536)
@@ -284,7 +295,8 @@ def test_fp8_zero_groups_and_options(lib):
 @pytest.mark.parametrize("plan", QK_PLANS)
 def test_qk_every_plan(lib, plan):
     for T, W, q_size, kv_size in ((1, 8, 6144, 1024), (5, 8, 6144, 1024), (3, 1, 64, 32),
-                                  (7, 2, 256, 128), (9, 16, 2048, 128), (33, 4, 512, 64)):
+                                  (7, 2, 256, 128), (9, 16, 2048, 128), (33, 4, 512, 64),
+                                  (600, 8, 6144, 1024)):   # several tokens per persistent CTA
         inp = wl.make_qk_inputs(wl.QK, T, W=W, q_size=q_size, kv_size=kv_size, seed=T + W + q_size)
         check_qk(lib, inp, plan=plan)
 
