@@ -314,6 +314,8 @@ int run_norm(const void *const *partials, const void *residual, const void *weig
     p.W = W;
     p.inv_H = 1.0 / (double)H;
     p.eps = (double)eps;
+    p.inv_Hf = (float)p.inv_H;
+    p.epsf = eps;
     p.gemma = gemma ? 1 : 0;
 
     p.withhold_row = -1;
