@@ -359,39 +359,109 @@ def plan_of(ar, call):
     return ar.ar_plan_query(1 if w.fp8 else 0, T, w.H, w.W, wl.DTYPE_CODE[dt])
 
 
+_E2E_IN = {"qk": ("qkv", "qw", "kw"), "norm": ("parts", "res", "w")}
+_E2E_OUT = {"qk": ("q_out", "k_out"), "norm": ("out", "rout", "q", "s")}
+
+
+def _carve_into(b, names, slab, off):
+    """Replace b's tensors `names` by views of `slab` from byte `off` on
+    (256-byte aligned each, contents copied); returns the next offset."""
+    for name in names:
+        v = getattr(b, name, None)
+        if v is None:
+            continue
+        ts = v if isinstance(v, list) else [v]
+        views = []
+        for t in ts:
+            nb = t.numel() * t.element_size()
+            view = slab[off:off + nb].view(t.dtype).view(t.shape)
+            view.copy_(t)
+            views.append(view)
+            off += (nb + 255) // 256 * 256
+        setattr(b, name, views if isinstance(v, list) else views[0])
+    return off
+
+
+def _e2e_sizes(b):
+    kind = "qk" if b.call[0] == "qk" else "norm"
+    def size(names, padded):
+        n = 0
+        for name in names:
+            v = getattr(b, name, None)
+            for t in ([] if v is None else v if isinstance(v, list) else [v]):
+                nb = t.numel() * t.element_size()
+                n += (nb + 255) // 256 * 256 if padded else nb
+        return n
+    return kind, size(_E2E_IN[kind], True), size(_E2E_OUT[kind], True), \
+        size(_E2E_IN[kind], False), size(_E2E_OUT[kind], False)
+
+
 def e2e_measure(ar, device, stream, calls, steps):
-    """Host buffers in, host buffers out, through the public call."""
+    """End to end through the public calls with host buffers.  Every step
+    copies all of its inputs from pinned host memory (one contiguous staging
+    area, one host-to-device copy) and reads all of its results back into
+    pinned host memory (one device-to-host copy).  Two device buffer sets
+    alternate, so that step k+1's input copy and step k's result copy run on
+    the two copy engines while step k computes (copy-in, compute and
+    copy-out streams ordered by events).  Returns (seconds for `steps`
+    steps, input bytes per step, output bytes per step)."""
     import torch
-    host_in, host_out, dev = [], [], []
-    for call in calls:
-        b = CallBuffers(call, device)
-        hin = [t.cpu().pin_memory() for t in b.inputs()]
-        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in b.outputs()]
-        host_in.append(hin)
-        host_out.append(hout)
-        dev.append(b)
-    h2d = sum(t.numel() * t.element_size() for hin in host_in for t in hin)
-    d2h = sum(t.numel() * t.element_size() for hout in host_out for t in hout)
+    sets = []
+    for _ in range(2):
+        bufs = [CallBuffers(call, device) for call in calls]
+        sizes = [_e2e_sizes(b) for b in bufs]
+        in_bytes = sum(x[1] for x in sizes)
+        out_bytes = sum(x[2] for x in sizes)
+        din = torch.empty(in_bytes, dtype=torch.uint8, device=device)
+        dout = torch.empty(out_bytes, dtype=torch.uint8, device=device)
+        oi = oo = 0
+        for b, (kind, _, _, _, _) in zip(bufs, sizes):
+            oi = _carve_into(b, _E2E_IN[kind], din, oi)
+            oo = _carve_into(b, _E2E_OUT[kind], dout, oo)
+        sets.append((bufs, din, dout))
+    h2d = sum(_e2e_sizes(b)[3] for b in sets[0][0])
+    d2h = sum(_e2e_sizes(b)[4] for b in sets[0][0])
+    host_in = sets[0][1].cpu().pin_memory()
+    host_out = torch.empty(sets[0][2].numel(), dtype=torch.uint8, pin_memory=True)
+    torch.cuda.synchronize()
 
-    def one_step():
-        for b, hin, hout in zip(dev, host_in, host_out):
-            for d, h in zip(b.inputs(), hin):
-                d.copy_(h, non_blocking=True)
-            b.run(ar)
-            for h, d in zip(hout, b.outputs()):
-                h.copy_(d, non_blocking=True)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
+    computed = [ev(), ev()]
+    copied_out = [ev(), ev()]
+    ready = [ev(), ev()]
+    for e in computed + copied_out:
+        e.record(stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            one_step()
-        torch.cuda.synchronize()
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-        for _ in range(steps):
-            one_step()
-        end.record(stream)
+    def one_step(k):
+        bufs, din, dout = sets[k & 1]
+        s_in.wait_event(computed[k & 1])             # step k-2 is done with these inputs
+        with torch.cuda.stream(s_in):
+            din.copy_(host_in, non_blocking=True)
+        ready[k & 1].record(s_in)
+        stream.wait_event(ready[k & 1])
+        stream.wait_event(copied_out[k & 1])         # step k-2's results have left
+        with torch.cuda.stream(stream):
+            for b in bufs:
+                b.run(ar)
+        computed[k & 1].record(stream)
+        s_out.wait_event(computed[k & 1])
+        with torch.cuda.stream(s_out):
+            host_out.copy_(dout, non_blocking=True)
+        copied_out[k & 1].record(s_out)
+
+    for k in range(2):
+        one_step(k)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for k in range(steps):
+        one_step(k)
+    end.record(s_out)
+    s_in.wait_stream(s_out)
     end.synchronize()
+    torch.cuda.synchronize()
     return start.elapsed_time(end) / 1e3, h2d, d2h
 
 
