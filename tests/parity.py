@@ -1,7 +1,7 @@
 """Comparison rules between the CUDA path and the fp64 oracle, and helpers
 that run one workload instance through both.
 
-Tolerances (fixed by the task's numeric contract, derived in the design doc):
+Tolerances:
   * 16-bit y: per element |g - o| <= 4e-3 |o|, or g within one unit in the
     last place of RNE(o) (covers exact zeros and fp16 subnormals where
     rounding alone exceeds 4e-3);
