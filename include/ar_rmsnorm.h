@@ -163,9 +163,14 @@ AR_API int ar_add_rmsnorm_quant_fp8_group(const void *const *partials,
  *           slice)
  * q_out     host array of W device pointers, each [T, qs], dense
  * k_out     host array of W device pointers, each [T, ks], dense
+ *           In-place form: q_out[w] == qkv[w] and k_out[w] == qkv[w] + qs
+ *           (elements) for every w.  The outputs then have qkv's row stride
+ *           and overwrite the q and k columns; v is untouched.  A call
+ *           that uses this form for some shards but not all returns
+ *           AR_EINVAL.  (Each row is read completely before it is written.)
  * Requirements: 1 <= W <= AR_MAX_W, q_size and kv_size positive multiples
  * of W with qs and ks multiples of 8, qs + ks <= AR_MAX_H, pointers 16-byte
- * aligned, outputs not overlapping inputs.
+ * aligned; apart from the in-place form, outputs do not overlap inputs.
  */
 AR_API int qk_norm_sharded(const void *const *qkv, const void *q_weight,
                     const void *k_weight, void *const *q_out,

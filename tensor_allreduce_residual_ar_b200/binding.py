@@ -147,10 +147,20 @@ def ar_add_rmsnorm_quant_fp8_group(partials, residual, weight, out_fp8, scales, 
 
 def qk_norm_sharded(qkv, q_weight, k_weight, q_out, k_out, q_size: int, kv_size: int,
                     eps: float = 1e-6, stream=None) -> None:
-    """Sharded QK-norm over W = len(qkv) shards, each [T, q_size/W + 2*kv_size/W]."""
+    """Sharded QK-norm over W = len(qkv) shards, each [T, q_size/W + 2*kv_size/W].
+    q_out[w] / k_out[w] are dense [T, q_size/W] / [T, kv_size/W] tensors, or,
+    for the in-place form, the views qkv[w][:, :qs] and qkv[w][:, qs:qs+ks]."""
     W = len(qkv)
-    row = q_size // W + 2 * (kv_size // W)
+    qs, ks = q_size // W, kv_size // W
+    row = qs + 2 * ks
     T = _rows(qkv[0], row)
+    for w in range(W):
+        for out, off, width in ((q_out[w], 0, qs), (k_out[w], qs, ks)):
+            inplace = (out.data_ptr() == qkv[w].data_ptr() + off * qkv[w].element_size()
+                       and out.dim() == 2 and out.shape == (T, width) and out.stride() == (row, 1))
+            if not inplace and not (out.is_contiguous() and out.numel() == T * width):
+                raise ValueError(f"shard {w}: output must be a dense [T, {width}] tensor or the "
+                                 f"in-place view of qkv[{w}]")
     lib = load_library()
     _check("qk_norm_sharded", lib.qk_norm_sharded(
         _ptrs(qkv), _ptr(q_weight), _ptr(k_weight), _ptrs(q_out), _ptrs(k_out), T, int(q_size),

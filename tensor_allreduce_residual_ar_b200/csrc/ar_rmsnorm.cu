@@ -430,6 +430,14 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
         if (!aligned(qkv[w], 16) || !aligned(q_out[w], 16) || !aligned(k_out[w], 16)) return AR_EALIGN;
     }
     if (!aligned(q_weight, 16) || !aligned(k_weight, 16)) return AR_EALIGN;
+    // in-place form: q_out[w] == qkv[w] and k_out[w] == qkv[w] + qs elements
+    // for every shard; the outputs then have qkv's row stride
+    const bool inplace = q_out[0] == qkv[0];
+    for (int w = 0; w < W; ++w) {
+        const char *base = static_cast<const char *>(qkv[w]);
+        const bool ip = q_out[w] == qkv[w] && static_cast<const char *>(k_out[w]) == base + qs * 2;
+        if (ip != inplace) return AR_EINVAL;
+    }
     if (T == 0) return AR_OK;
 
     DevInfo di;
@@ -451,6 +459,8 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
     p.qsp = (int)(qs / 8);
     p.ksp = (int)(ks / 8);
     p.row_packs = p.qsp + 2 * p.ksp;
+    p.q_stride = inplace ? p.row_packs : p.qsp;
+    p.k_stride = inplace ? p.row_packs : p.ksp;
     p.inv_q = (float)(1.0 / (double)q_size);
     p.inv_k = (float)(1.0 / (double)kv_size);
     p.eps = eps;

@@ -33,3 +33,14 @@ def lib(cuda_device):
     import tensor_allreduce_residual_ar_b200 as ar
     ar.load_library()
     return ar
+
+
+@pytest.fixture(autouse=True)
+def _clear_forced_plans(request):
+    """A plan forced by one test never leaks into the next: after every test
+    that used the library, every variant goes back to the plan table."""
+    yield
+    if "lib" in request.fixturenames:
+        import tensor_allreduce_residual_ar_b200 as ar
+        for variant in (0, 1, 2):
+            ar.ar_plan_force(variant, 0)

@@ -175,6 +175,27 @@ def test_plan_table_load_and_reject(clib, tmp_path):
     assert clib.ar_plan_load(None) == OK and clib.ar_plan_table_size() == 0
 
 
+def test_qk_inplace_form_must_cover_every_shard(clib):
+    """In-place QK (q_out[w] == qkv[w], k_out[w] == qkv[w] + qs) is all or
+    nothing; a mixture is an argument error, found before any device access."""
+    W, qs, ks = 2, 64, 32
+    base = [0x100000, 0x200000]
+    qkv = _ptrs(*base)
+    inplace_q = _ptrs(*base)
+    inplace_k = _ptrs(*[b + 2 * qs for b in base])
+    dense_q = _ptrs(0x300000, 0x400000)
+    dense_k = _ptrs(0x500000, 0x600000)
+    f = clib.qk_norm_sharded
+    # T = 0: validated, nothing launched
+    assert f(qkv, C_, D, inplace_q, inplace_k, 0, W * qs, W * ks, W, 1e-6, 0, None) == OK
+    assert f(qkv, C_, D, dense_q, dense_k, 0, W * qs, W * ks, W, 1e-6, 0, None) == OK
+    mixed_q = _ptrs(base[0], 0x400000)
+    mixed_k = _ptrs(base[0] + 2 * qs, 0x600000)
+    assert f(qkv, C_, D, mixed_q, mixed_k, 0, W * qs, W * ks, W, 1e-6, 0, None) == EINVAL
+    bad_k = _ptrs(base[0] + 2 * qs + 16, base[1] + 2 * qs)
+    assert f(qkv, C_, D, inplace_q, bad_k, 0, W * qs, W * ks, W, 1e-6, 0, None) == EINVAL
+
+
 def test_plan_force(clib):
     q = ctypes.c_int(-1)
     assert clib.ar_plan_force(0, 11) == EINVAL      # QK plan for the norm variant

@@ -301,6 +301,43 @@ def test_qk_every_plan(lib, plan):
         check_qk(lib, inp, plan=plan)
 
 
+@pytest.mark.parametrize("plan", QK_PLANS)
+def test_qk_in_place(lib, plan):
+    """In-place form: q_out[w] / k_out[w] are the q / k column views of
+    qkv[w]; those columns are overwritten with the normalised values and
+    the v columns stay bit-identical."""
+    for T, dtype in ((5, "bf16"), (300, "fp16")):
+        inp = wl.make_qk_inputs(wl.QK, T, dtype, seed=500 + T)
+        W, qs, ks = inp.W, inp.q_size // inp.W, inp.kv_size // inp.W
+        qkv = [x.to("cuda").clone() for x in inp.qkv]
+        v_before = [x[:, qs + ks:].clone() for x in qkv]
+        assert lib.ar_plan_force(2, plan) == 0
+        try:
+            lib.qk_norm_sharded(qkv, inp.q_weight.to("cuda"), inp.k_weight.to("cuda"),
+                                [x[:, :qs] for x in qkv], [x[:, qs:qs + ks] for x in qkv],
+                                inp.q_size, inp.kv_size, eps=inp.eps)
+            torch.cuda.synchronize()
+        finally:
+            lib.ar_plan_force(2, 0)
+        q64, k64 = P.oracle_qk(inp)
+        for w in range(W):
+            P.check_y(P.to_bits(qkv[w][:, :qs].contiguous()), q64[w], dtype, f"q[{w}]")
+            P.check_y(P.to_bits(qkv[w][:, qs:qs + ks].contiguous()), k64[w], dtype, f"k[{w}]")
+            assert torch.equal(qkv[w][:, qs + ks:], v_before[w]), "v must not be modified"
+
+
+def test_qk_rejects_strided_outputs(lib):
+    inp = wl.make_qk_inputs(wl.QK, 4, seed=77)
+    W, qs, ks = inp.W, inp.q_size // inp.W, inp.kv_size // inp.W
+    qkv = [x.to("cuda") for x in inp.qkv]
+    wide = torch.empty((4, 2 * qs), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        lib.qk_norm_sharded(qkv, inp.q_weight.to("cuda"), inp.k_weight.to("cuda"),
+                            [wide[:, :qs]] * W, [torch.empty((4, ks), dtype=torch.bfloat16,
+                                                              device="cuda")] * W,
+                            inp.q_size, inp.kv_size, eps=inp.eps)
+
+
 def test_qk_fp16(lib):
     inp = wl.make_qk_inputs(wl.QK, 17, "fp16", seed=3)
     check_qk(lib, inp)
