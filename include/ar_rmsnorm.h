@@ -131,7 +131,7 @@ AR_API int ar_add_rmsnorm(const void *const *partials, const void *residual,
  *   out_fp8[t,h]  = e4m3fn_RNE_satfinite(y[t,h] / scales[t,g]),
  *                   0 for every element when amax == 0
  * out_fp8       [T, H] bytes, OCP e4m3fn codes (1-4-3, bias 7, max 448)
- * scales        [T, H/group] fp32, row-major
+ * scales        [T, H/group] fp32, row-major (any layout: the _strided call)
  * out_y         [T, H] in `dtype` (RNE of y) or NULL
  * residual_out  [T, H] in `dtype` or NULL, as in ar_add_rmsnorm
  * group         must be 128; H must be a multiple of it
@@ -144,6 +144,24 @@ AR_API int ar_add_rmsnorm_quant_fp8_group(const void *const *partials,
                                    void *residual_out, int64_t T, int64_t H,
                                    int W, int group, float eps, int gemma,
                                    int dtype, cudaStream_t stream);
+
+/*
+ * ar_add_rmsnorm_quant_fp8_group_strided -- as ar_add_rmsnorm_quant_fp8_group
+ * with any scales layout: scales[t, g] lives at
+ *   scales[t * scale_stride_t + g * scale_stride_g]   (elements).
+ * Row-major [T, H/group] is (H/group, 1); the transposed [H/group, T] layout
+ * is (1, T).  The strides must be >= 0 and give every (t, g) its own slot
+ * (row-major-like: stride_g >= 1 and stride_t >= (H/group) * stride_g, or
+ * column-major-like: stride_t >= 1 and stride_g >= T * stride_t; one of
+ * them may be anything when T or H/group is 1), else AR_EINVAL.
+ */
+AR_API int ar_add_rmsnorm_quant_fp8_group_strided(const void *const *partials,
+                                   const void *residual, const void *weight,
+                                   void *out_fp8, float *scales,
+                                   int64_t scale_stride_t, int64_t scale_stride_g,
+                                   void *out_y, void *residual_out, int64_t T,
+                                   int64_t H, int W, int group, float eps,
+                                   int gemma, int dtype, cudaStream_t stream);
 
 /*
  * qk_norm_sharded -- MiniMax-style QK-norm over W tensor-parallel shards.

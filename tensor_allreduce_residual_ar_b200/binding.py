@@ -54,6 +54,9 @@ def load_library():
         lib.ar_add_rmsnorm_quant_fp8_group.restype = i32
         lib.ar_add_rmsnorm_quant_fp8_group.argtypes = [PP, P, P, P, P, P, P, i64, i64, i32, i32,
                                                        f32, i32, i32, P]
+        lib.ar_add_rmsnorm_quant_fp8_group_strided.restype = i32
+        lib.ar_add_rmsnorm_quant_fp8_group_strided.argtypes = [PP, P, P, P, P, i64, i64, P, P, i64,
+                                                               i64, i32, i32, f32, i32, i32, P]
         lib.qk_norm_sharded.restype = i32
         lib.qk_norm_sharded.argtypes = [PP, P, P, PP, PP, i64, i64, i64, i32, f32, i32, P]
         lib.ar_plan_query.restype = i32
@@ -134,15 +137,24 @@ def ar_add_rmsnorm_quant_fp8_group(partials, residual, weight, out_fp8, scales, 
                                    residual_out=None, eps: float = 1e-6, gemma: bool = False,
                                    group: int = 128, stream=None) -> None:
     """As ar_add_rmsnorm, then per-group e4m3 codes ``out_fp8`` (uint8 or
-    float8_e4m3fn [..., H]) and fp32 ``scales`` [..., H/group]; the 16-bit y
-    goes to ``out_y`` when given."""
+    float8_e4m3fn [..., H]) and fp32 ``scales``; the 16-bit y goes to
+    ``out_y`` when given.  ``scales`` is a [T, H/group] tensor of any strides
+    (e.g. the transpose of a [H/group, T] buffer) or a contiguous
+    [..., H/group] tensor."""
     H = weight.shape[-1]
     T = _rows(partials[0], H)
+    G = H // group if group > 0 else 0
+    if scales.dim() == 2 and tuple(scales.shape) == (T, G):
+        s_t, s_g = scales.stride()
+    elif scales.is_contiguous() and scales.numel() == T * G:
+        s_t, s_g = G, 1
+    else:
+        raise ValueError(f"scales must be [T, {G}] (any strides) or contiguous [..., {G}]")
     lib = load_library()
-    _check("ar_add_rmsnorm_quant_fp8_group", lib.ar_add_rmsnorm_quant_fp8_group(
-        _ptrs(partials), _ptr(residual), _ptr(weight), _ptr(out_fp8), _ptr(scales), _ptr(out_y),
-        _ptr(residual_out), T, H, len(partials), int(group), float(eps), int(bool(gemma)),
-        _dtype(weight), _stream(stream)))
+    _check("ar_add_rmsnorm_quant_fp8_group", lib.ar_add_rmsnorm_quant_fp8_group_strided(
+        _ptrs(partials), _ptr(residual), _ptr(weight), _ptr(out_fp8), _ptr(scales), s_t, s_g,
+        _ptr(out_y), _ptr(residual_out), T, H, len(partials), int(group), float(eps),
+        int(bool(gemma)), _dtype(weight), _stream(stream)))
 
 
 def qk_norm_sharded(qkv, q_weight, k_weight, q_out, k_out, q_size: int, kv_size: int,

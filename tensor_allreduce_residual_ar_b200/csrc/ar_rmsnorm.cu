@@ -293,8 +293,9 @@ int validate_norm_common(const void *const *partials, const void *residual, cons
 }
 
 int run_norm(const void *const *partials, const void *residual, const void *weight, void *out,
-             void *residual_out, uint8_t *out_fp8, float *scales, int64_t T, int64_t H, int W,
-             float eps, int gemma, int dtype, bool fp8, cudaStream_t stream) {
+             void *residual_out, uint8_t *out_fp8, float *scales, int64_t s_row, int64_t s_grp,
+             int64_t T, int64_t H, int W, float eps, int gemma, int dtype, bool fp8,
+             cudaStream_t stream) {
     DevInfo di;
     int st = device_info(di);
     if (st != AR_OK) return st;
@@ -309,6 +310,8 @@ int run_norm(const void *const *partials, const void *residual, const void *weig
     p.residual_out = residual_out;
     p.out_fp8 = out_fp8;
     p.scales = scales;
+    p.s_row = s_row;
+    p.s_grp = s_grp;
     p.T = T;
     p.P = (int)(H / 8);
     p.W = W;
@@ -393,23 +396,46 @@ int ar_add_rmsnorm(const void *const *partials, const void *residual, const void
     if (out == nullptr) return AR_EINVAL;
     if (!aligned(out, 16)) return AR_EALIGN;
     if (T == 0) return AR_OK;
-    return run_norm(partials, residual, weight, out, residual_out, nullptr, nullptr, T, H, W, eps,
-                    gemma, dtype, false, stream);
+    return run_norm(partials, residual, weight, out, residual_out, nullptr, nullptr, 0, 0, T, H, W,
+                    eps, gemma, dtype, false, stream);
+}
+
+int ar_add_rmsnorm_quant_fp8_group_strided(const void *const *partials, const void *residual,
+                                           const void *weight, void *out_fp8, float *scales,
+                                           int64_t scale_stride_t, int64_t scale_stride_g,
+                                           void *out_y, void *residual_out, int64_t T, int64_t H,
+                                           int W, int group, float eps, int gemma, int dtype,
+                                           cudaStream_t stream) {
+    int st = validate_norm_common(partials, residual, weight, residual_out, T, H, W, eps, dtype);
+    if (st != AR_OK) return st;
+    if (out_fp8 == nullptr || scales == nullptr) return AR_EINVAL;
+    if (group != 128 || H % group != 0) return AR_EINVAL;
+    // every (row, group) must own a distinct scale slot
+    {
+        const __int128 G = H / group, st_t = scale_stride_t, st_g = scale_stride_g;
+        if (st_t < 0 || st_g < 0) return AR_EINVAL;
+        bool ok;
+        if (G == 1 && T <= 1) ok = true;
+        else if (G == 1) ok = st_t >= 1;
+        else if (T <= 1) ok = st_g >= 1;
+        else ok = (st_g >= 1 && st_t >= G * st_g) || (st_t >= 1 && st_g >= (__int128)T * st_t);
+        if (!ok) return AR_EINVAL;
+    }
+    if (!aligned(out_fp8, 16) || !aligned(scales, 4)) return AR_EALIGN;
+    if (out_y && !aligned(out_y, 16)) return AR_EALIGN;
+    if (T == 0) return AR_OK;
+    return run_norm(partials, residual, weight, out_y, residual_out, (uint8_t *)out_fp8, scales,
+                    scale_stride_t, scale_stride_g, T, H, W, eps, gemma, dtype, true, stream);
 }
 
 int ar_add_rmsnorm_quant_fp8_group(const void *const *partials, const void *residual,
                                    const void *weight, void *out_fp8, float *scales, void *out_y,
                                    void *residual_out, int64_t T, int64_t H, int W, int group,
                                    float eps, int gemma, int dtype, cudaStream_t stream) {
-    int st = validate_norm_common(partials, residual, weight, residual_out, T, H, W, eps, dtype);
-    if (st != AR_OK) return st;
-    if (out_fp8 == nullptr || scales == nullptr) return AR_EINVAL;
-    if (group != 128 || H % group != 0) return AR_EINVAL;
-    if (!aligned(out_fp8, 16) || !aligned(scales, 4)) return AR_EALIGN;
-    if (out_y && !aligned(out_y, 16)) return AR_EALIGN;
-    if (T == 0) return AR_OK;
-    return run_norm(partials, residual, weight, out_y, residual_out, (uint8_t *)out_fp8, scales, T, H,
-                    W, eps, gemma, dtype, true, stream);
+    const int64_t groups = group > 0 ? H / group : 0;
+    return ar_add_rmsnorm_quant_fp8_group_strided(partials, residual, weight, out_fp8, scales,
+                                                  groups, 1, out_y, residual_out, T, H, W, group,
+                                                  eps, gemma, dtype, stream);
 }
 
 int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_weight,

@@ -25,6 +25,8 @@ def clib():
     lib.ar_add_rmsnorm.argtypes = [PP, P, P, P, P, i64, i64, i32, f32, i32, i32, P]
     lib.ar_add_rmsnorm_quant_fp8_group.argtypes = [PP, P, P, P, P, P, P, i64, i64, i32, i32, f32,
                                                    i32, i32, P]
+    lib.ar_add_rmsnorm_quant_fp8_group_strided.argtypes = [PP, P, P, P, P, i64, i64, P, P, i64, i64,
+                                                           i32, i32, f32, i32, i32, P]
     lib.qk_norm_sharded.argtypes = [PP, P, P, PP, PP, i64, i64, i64, i32, f32, i32, P]
     lib.ar_plan_query.argtypes = [i32, i64, i64, i32, i32, ctypes.POINTER(ctypes.c_int)]
     lib.ar_plan_load.argtypes = [ctypes.c_char_p]
@@ -108,6 +110,24 @@ def test_fp8_argument_errors(clib):
     assert call(s=E + 2) == EALIGN
     assert call(y=A + 4) == EALIGN
     assert call(s=E + 4, T=0) == OK         # scales need only 4-byte alignment
+
+
+def test_fp8_scale_strides(clib):
+    """Scale layouts: every (row, group) needs its own slot; checked before
+    any device access."""
+    parts = _ptrs(A, B)
+    f = clib.ar_add_rmsnorm_quant_fp8_group_strided
+    def call(st, sg, T=5, H=256):              # G = 2 groups
+        return f(parts, None, C_, D, E, st, sg, None, None, T, H, 2, 128, 1e-6, 0, 0, None)
+    assert call(1, 1) == EINVAL                # rows overlap groups
+    assert call(-2, 1) == EINVAL
+    assert call(2, 0) == EINVAL
+    assert call(1, 4) == EINVAL                # column-major needs stride_g >= T
+    assert call(0, 1) == EINVAL
+    assert call(2, 1, T=0) == OK               # row-major
+    assert call(1, 5, T=0) == OK               # transposed [G, T]
+    assert call(0, 1, T=0) == OK               # no rows: the row stride is free
+    assert call(3, 0, T=0, H=128) == OK        # one group: the group stride is free
 
 
 def test_qk_argument_errors(clib):

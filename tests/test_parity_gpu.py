@@ -275,6 +275,30 @@ def test_fp8_every_plan_ragged(lib, plan):
         check_fp8(lib, inp, plan=plan)
 
 
+@pytest.mark.parametrize("plan", NORM_PLANS)
+def test_fp8_transposed_scales(lib, plan):
+    """Scales written through strides: the transpose of a [H/128, T] buffer
+    receives exactly the row-major scales, with the same codes and y; the
+    buffer's guard bands stay intact."""
+    T, H = 37, 5120
+    G = H // 128
+    inp = wl.make_norm_inputs(wl.FP8, T, W=4, H=H, seed=2024)
+    q0, s0, y0, r0 = run_fp8(lib, inp, plan=plan)
+    dev = "cuda"
+    parts = [p.to(dev) for p in inp.partials]
+    q = torch.empty((T, H), dtype=torch.uint8, device=dev)
+    st = Guarded((G, T), torch.float32, -7.0)
+    y = torch.empty((T, H), dtype=TD[inp.dtype], device=dev)
+    assert lib.ar_plan_force(1, plan) == 0
+    lib.ar_add_rmsnorm_quant_fp8_group(parts, inp.residual.to(dev), inp.weight.to(dev), q,
+                                       st.view.t(), y, None, eps=inp.eps, gemma=inp.gemma)
+    torch.cuda.synchronize()
+    assert st.guard_ok()
+    assert np.array_equal(st.view.t().cpu().numpy(), s0)
+    assert np.array_equal(q.cpu().numpy(), q0)
+    assert np.array_equal(P.to_bits(y), y0)
+
+
 def test_fp8_zero_groups_and_options(lib):
     T, H = 6, 512
     inp = wl.make_norm_inputs(wl.FP8, T, W=2, H=H, seed=99)
