@@ -340,11 +340,19 @@ def per_call_sweep(ar, device, stream, names, reps=20):
             graphs = capture_step_graphs(ar, [sets], stream)
             time_graphs(graphs, 2, stream)
             sec = time_graphs(graphs, reps, stream) / (reps * R)
-            rows.append({"T": call[2], "dtype": call[3], "us": round(sec * 1e6, 3),
-                         "GBps": round(nbytes / sec / 1e9, 1),
-                         "frac_of_measured": round(nbytes / sec / 1e9 / peak, 4),
-                         "frac_of_8TBps": round(nbytes / sec / 1e9 / NOMINAL_HBM_GBS, 4),
-                         "bytes": nbytes, "plan": plan_of(ar, call), "sets": R})
+            row = {"T": call[2], "dtype": call[3], "us": round(sec * 1e6, 3),
+                   "GBps": round(nbytes / sec / 1e9, 1),
+                   "frac_of_measured": round(nbytes / sec / 1e9 / peak, 4),
+                   "frac_of_8TBps": round(nbytes / sec / 1e9 / NOMINAL_HBM_GBS, 4),
+                   "bytes": nbytes, "plan": plan_of(ar, call), "sets": R}
+            if name in ("decode", "tiny"):
+                # the same call 64 times on one buffer set: inputs L2-resident
+                # (a latency figure, not a bandwidth one)
+                hot = capture_step_graphs(ar, [[base] * 64], stream)
+                time_graphs(hot, 2, stream)
+                row["us_hot_l2"] = round(time_graphs(hot, reps, stream) / (reps * 64) * 1e6, 3)
+                del hot
+            rows.append(row)
             del graphs, sets, base
             torch.cuda.empty_cache()
         out[name] = rows
