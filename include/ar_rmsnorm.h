@@ -214,7 +214,8 @@ typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_v
  * each), the grid sized to the clusters that fit at once.  PERSIST_AHEAD:
  * one CTA of up to 512 threads per row, persistent, each thread's next row
  * loaded into registers while the current one is finished (where the
- * register budget allows).  BULK: rows
+ * register budget allows); PERSIST_C2_AHEAD: the same with each row split
+ * over a cluster of 2 CTAs.  BULK: rows
  * staged into shared memory by bulk asynchronous copies.  QK_C<k>: one token
  * per cluster of k CTAs, shards split across the cluster; QK_PERSIST: one
  * CTA (at most 512 threads) per token, persistent grid with L2 prefetch;
@@ -230,6 +231,7 @@ enum {
     AR_PLAN_PERSIST512 = 7,
     AR_PLAN_PERSIST_C2 = 8,
     AR_PLAN_PERSIST_AHEAD = 9,
+    AR_PLAN_PERSIST_C2_AHEAD = 10,
     AR_PLAN_QK_C1 = 11,
     AR_PLAN_QK_C2 = 12,
     AR_PLAN_QK_C4 = 13,

@@ -34,7 +34,7 @@ std::vector<const Table *> g_retired;
 std::atomic<int> g_force[3] = {{0}, {0}, {0}};
 
 bool is_norm_plan(int id) {
-    return id >= AR_PLAN_ROWC1 && id <= AR_PLAN_PERSIST_AHEAD;
+    return id >= AR_PLAN_ROWC1 && id <= AR_PLAN_PERSIST_C2_AHEAD;
 }
 bool is_qk_plan(int id) { return id >= AR_PLAN_QK_C1 && id <= AR_PLAN_QK_PERSIST256; }
 
@@ -157,6 +157,7 @@ Geometry plan_geometry(int id) {
     case AR_PLAN_PERSIST512: return {1, true, 512, 2};
     case AR_PLAN_PERSIST_C2: return {2, true, 512, 2};
     case AR_PLAN_PERSIST_AHEAD: return {1, true, 512, 1};
+    case AR_PLAN_PERSIST_C2_AHEAD: return {2, true, 512, 1};
     case AR_PLAN_BULK: return {1, true, 512, 1};
     case AR_PLAN_QK_C1: return {1, false, 512, 1};
     case AR_PLAN_QK_C2: return {2, false, 512, 1};

@@ -24,7 +24,7 @@ from . import binding as ar
 from . import workloads as wl
 
 L2_BYTES = 126 * 1024 * 1024
-NORM_PLANS = (1, 2, 3, 4, 5, 6, 7, 8, 9)
+NORM_PLANS = (1, 2, 3, 4, 5, 6, 7, 8, 9, 10)
 QK_PLANS = (11, 12, 13, 14, 15, 16)
 T_MAX = 1 << 40
 

@@ -221,8 +221,8 @@ def test_plan_force(clib):
     assert clib.ar_plan_force(0, 11) == EINVAL      # QK plan for the norm variant
     assert clib.ar_plan_force(2, 1) == EINVAL
     assert clib.ar_plan_force(3, 1) == EINVAL
-    assert clib.ar_plan_force(0, 9) == OK           # PERSIST_AHEAD, the last norm plan
-    assert clib.ar_plan_force(0, 10) == EINVAL
+    assert clib.ar_plan_force(0, 10) == OK          # PERSIST_C2_AHEAD, the last norm plan
+    assert clib.ar_plan_force(0, 11) == EINVAL
     assert clib.ar_plan_force(2, 8) == EINVAL
     assert clib.ar_plan_force(2, 16) == OK          # QK_PERSIST256, the last QK plan
     assert clib.ar_plan_force(2, 17) == EINVAL
