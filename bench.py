@@ -253,7 +253,34 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and with whitespace runs collapsed
+    (string and character literals kept), so that editing a comment does not
+    count as a change of the kernels."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of what decides the timed kernels: the CUDA and host sources
+    (code only) and the plan table."""
     h = hashlib.sha256()
     for rel in ("tensor_allreduce_residual_ar_b200/csrc/kernels.cuh",
                 "tensor_allreduce_residual_ar_b200/csrc/ar_rmsnorm.cu",
@@ -261,8 +288,9 @@ def kernel_source_hash() -> str:
                 "tensor_allreduce_residual_ar_b200/plan_table.json"):
         p = os.path.join(ROOT, rel)
         if os.path.exists(p):
-            with open(p, "rb") as f:
-                h.update(f.read())
+            with open(p, encoding="utf-8") as f:
+                text = f.read()
+            h.update((text if rel.endswith(".json") else _code_only(text)).encode())
     return h.hexdigest()[:16]
 
 
