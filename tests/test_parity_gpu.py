@@ -422,20 +422,41 @@ def test_cancellation_sweep_around_certificate(lib, plan, dtype):
 
 
 @pytest.mark.parametrize("plan", NORM_PLANS)
-def test_fp8_rare_accuracy_paths(lib, plan):
-    """Crafted rows that drive the FP8 variant's rare paths:
-    row 0, group 0: the group maximum has a large partial-sum bound
-    (100 - 50 - 45 + 5 = 10, bound 65 > 4 * 10), so it is recomputed exactly
-    before the scale is formed; row 1: residual ~ -(sum of partials), so the
-    sum-of-squares error bound is large and the whole row is recomputed;
-    rows 2-3 ordinary."""
-    T, H, W = 4, 256, 3
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_fp8_rare_accuracy_paths(lib, plan, dtype):
+    """Crafted rows that drive the FP8 variant's rare paths.
+    row 0, elements 0-15: residual 1, partials k*tiny, -1, 0.  The fp32 sum
+    1 + k*tiny is not exact, so the sums rounded down and up differ and the
+    TwoSum recomputation must recover r = k*tiny (a plain fp32 sum gives 0).
+    row 1, group 1: values near 1e-30 (bf16; zero in fp16) while the rest of
+    the row is ordinary: the group scale falls below 2^-90 and the codes take
+    the IEEE division.
+    row 2, group 2: residual = -(sum of partials) exactly and weight -1: the
+    group is all zeros (scale 0, codes 0) with signed-zero outputs.
+    row 3: ordinary."""
+    T, H, W = 4, 512, 3
+    td = TD[dtype]
+    tiny = 2.0 ** -30 if dtype == "bf16" else 2.0 ** -24
     gen = torch.Generator().manual_seed(4242 + plan)
-    parts = [(0.5 * torch.randn(T, H, generator=gen)).to(torch.bfloat16) for _ in range(W)]
-    res = torch.randn(T, H, generator=gen).to(torch.bfloat16)
-    res[0, 0], parts[0][0, 0], parts[1][0, 0], parts[2][0, 0] = 100.0, -50.0, -45.0, 5.0
-    total = sum(p[1].double() for p in parts)
-    res[1] = (-total + 1e-3 * torch.randn(H, generator=gen).double()).to(torch.bfloat16)
-    w = (1.0 + 0.1 * torch.randn(H, generator=gen)).to(torch.bfloat16)
-    inp = wl.NormInputs(parts, res, w, T, H, W, "bf16", wl.eps32(1e-6), False, True)
-    check_fp8(lib, inp, plan=plan)
+    parts = [0.5 * torch.randn(T, H, generator=gen) for _ in range(W)]
+    res = torch.randn(T, H, generator=gen)
+    w = 1.0 + 0.1 * torch.randn(H, generator=gen)
+    k = torch.arange(1, 17, dtype=torch.float32)
+    res[0, :16], parts[0][0, :16], parts[1][0, :16], parts[2][0, :16] = 1.0, k * tiny, -1.0, 0.0
+    for x in [res] + parts:
+        x[1, 128:256] *= 1e-30
+    g2 = slice(256, 384)
+    for n, x in enumerate(parts):
+        x[2, g2] = torch.randint(-8, 9, (128,), generator=gen).float() * (n + 1)
+    res[2, g2] = -(parts[0][2, g2] + parts[1][2, g2] + parts[2][2, g2])
+    w[g2] = -1.0
+    parts = [x.to(td) for x in parts]
+    inp = wl.NormInputs(parts, res.to(td), w.to(td), T, H, W, dtype, wl.eps32(1e-6), False, True)
+    q, s, y, r = run_fp8(lib, inp, plan=plan)
+    o = P.oracle_norm(inp)
+    P.check_fp8(q, s, o["y"])
+    P.check_y(y, o["y"], dtype)
+    P.check_res(r, o["r"], dtype)
+    exact = (k * tiny).to(td).view(torch.int16).numpy()
+    assert np.array_equal(r[0, :16].astype(np.int16), exact), "TwoSum recovery of r = k*tiny"
+    assert np.all(s[2, 2] == 0.0) and np.all(q[2, 256:384] & 0x7F == 0)
