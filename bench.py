@@ -685,21 +685,25 @@ def run_ours(args):
             "clocks": sampler.summary()}
 
     del graphs
-    if not args.no_sweep and rank == 0:
+    # Every collective is done: the ranks part here, so that rank 0's
+    # sweep and oracle timing below (no collectives, a minute or more) keep
+    # no other rank waiting in a barrier against the group's timeout.
+    if world > 1:
+        barrier(device)
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    if not args.no_sweep:
         names = ["tiny", "decode", "prefill", "fp8", "qk"] if args.sweep == "all" else \
             [n for n in args.sweep.split(",") if n]
         line["sweep"] = per_call_sweep(ar, device, stream, names)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline:
         el_c, n_c, sb = oracle_sample(calls, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(sb * n_c / el_c / 1e9, 5), "unit": "GB/s", "cores": 1,
                                 "kind": "oracle",
                                 "sample": f"{n_c} full steps of the {args.workload} workload "
                                           f"({len(calls)} calls each) in {el_c:.1f} s, single-threaded C fp64"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        barrier(device)
-        dist.destroy_process_group()
+    print(json.dumps(line), flush=True)
     return 0
 
 
