@@ -206,20 +206,28 @@ AR_API int qk_norm_sharded(const void *const *qkv, const void *q_weight,
  */
 typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_variant;
 
-/* Plan ids.  ROWC<k>: one row per cluster of k CTAs (sum of squares combined
- * through distributed shared memory).  PERSIST / PERSIST512: one CTA of at
- * most 256 / 512 threads per row, grid sized to the SM count x occupancy,
- * rows looped, each CTA's next row bulk-prefetched into L2.  PERSIST_C2: the
- * same with each row split over a cluster of 2 CTAs (at most 512 threads
- * each), the grid sized to the clusters that fit at once.  PERSIST_AHEAD:
- * one CTA of up to 512 threads per row, persistent, each thread's next row
- * loaded into registers while the current one is finished (where the
- * register budget allows); PERSIST_C2_AHEAD: the same with each row split
- * over a cluster of 2 CTAs.  BULK: rows
- * staged into shared memory by bulk asynchronous copies.  QK_C<k>: one token
- * per cluster of k CTAs, shards split across the cluster; QK_PERSIST: one
- * CTA (at most 512 threads) per token, persistent grid with L2 prefetch;
- * QK_PERSIST256: the same with at most 256 threads (more packs per thread). */
+/* Plan ids.
+ *   ROWC<k>           one row per cluster of k CTAs; the sum of squares is
+ *                     combined through distributed shared memory.
+ *   PERSIST           one CTA of at most 256 threads per row; persistent grid
+ *                     (SM count x occupancy), rows looped, each CTA's next
+ *                     row bulk-prefetched into L2.
+ *   PERSIST512        the same with at most 512 threads, two CTAs per SM.
+ *   PERSIST_C2        the same with each row split over a cluster of 2 CTAs;
+ *                     the grid is the number of clusters that fit at once.
+ *   PERSIST_AHEAD     one CTA of at most 512 threads per row, persistent; each
+ *                     thread's next row is loaded into registers while the
+ *                     current one is finished (where the register budget
+ *                     allows).
+ *   PERSIST_C2_AHEAD  the same with each row split over a cluster of 2 CTAs.
+ *   BULK              rows staged into shared memory by bulk asynchronous
+ *                     copies.
+ *   QK_C<k>           one token per cluster of k CTAs, shards split across
+ *                     the cluster.
+ *   QK_PERSIST        one CTA of at most 512 threads per token, persistent
+ *                     grid with L2 prefetch.
+ *   QK_PERSIST256     the same with at most 256 threads (more packs per
+ *                     thread). */
 enum {
     AR_PLAN_AUTO = 0,
     AR_PLAN_ROWC1 = 1,
