@@ -235,6 +235,25 @@ def test_plan_force(clib):
     assert clib.ar_plan_query(2, 1, 7168, 8, 0, ctypes.byref(q)) == OK and 11 <= q.value <= 14
 
 
+def test_plan_ids_agree_across_header_library_tuner_and_tests(clib):
+    """Every plan id the header names is accepted for its variant and
+    nothing else is; the tuner and the every-plan GPU tests cover exactly
+    those ids."""
+    import re
+    from tensor_allreduce_residual_ar_b200 import tune
+    import test_parity_gpu as tp
+    hdr = open(os.path.join(ROOT, "include", "ar_rmsnorm.h")).read()
+    ids = {name: int(v) for name, v in re.findall(r"AR_PLAN_(\w+) = (\d+)", hdr)}
+    qk = {v for n, v in ids.items() if n.startswith("QK_")}
+    norm = {v for n, v in ids.items() if v != 0 and not n.startswith("QK_")}
+    for variant, valid in ((0, norm), (1, norm), (2, qk)):
+        accepted = {pid for pid in range(1, 40) if clib.ar_plan_force(variant, pid) == OK}
+        clib.ar_plan_force(variant, 0)
+        assert accepted == valid, (variant, sorted(accepted), sorted(valid))
+    assert set(tune.NORM_PLANS) == norm and set(tune.QK_PLANS) == qk
+    assert set(tp.NORM_PLANS) == norm and set(tp.QK_PLANS) == qk
+
+
 def test_builtin_rule_is_capture_static(clib):
     """Same arguments, same plan, however often asked (no state, no data)."""
     q1, q2 = ctypes.c_int(-1), ctypes.c_int(-1)
