@@ -1,26 +1,29 @@
 """Benchmark of the fused W-way reduce + residual add + RMSNorm library.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|tiny|prefill|fp8|qk] [--no-sweep]
+                    [--workload prefill|decode|tiny|fp8|qk] [--no-sweep]
 
-One step = one pass over every call of the chosen workload (default: the
-decode window, T in {1,2,4,8,16,32,64,80} x {bf16, fp16}, H=8192, W=4,
-Gemma RMSNorm: 16 calls), each call through the C ABI, the whole step
-captured once in a CUDA graph per rotating buffer set and replayed.  Buffer
-sets rotate so the data a step touches was last touched more than 2x L2
-ago (cold HBM), or the inputs alone exceed L2.  Rank 0 prints one JSON line.
+One step = one pass over every call of the chosen workload, each call
+through the C ABI, the whole step captured once in a CUDA graph per rotating
+buffer set and replayed.  The default workload is the largest single-GPU
+configuration of the fused reduce + add + RMSNorm: prefill, dead residual,
+T=8192, H=4096, W=8 bf16 partials (671 MB of algorithmic traffic per call,
+inputs larger than L2).  Buffer sets rotate so the data a step touches was
+last touched more than 2x L2 ago (cold HBM), or the inputs alone exceed L2.
+Rank 0 prints one JSON line, last; the per-call sweep of every workload is
+printed as plain text lines before it.
 
 value       achieved GB/s = algorithmic bytes of all ranks' steps / max-over-ranks
             device time (CUDA events around exactly K steps)
 e2e         the same metric through the same public call with host buffers:
             pinned host -> device copies of every input, the call, and the
             device -> host copy of every output, all inside the timed region
-roofline    the step's kernels against the measured HBM copy bandwidth
+roofline    the step's kernel against the measured HBM copy bandwidth
 cpu_baseline / --impl reference
-            the fp64 CPU oracle, single-threaded, on a bounded sample of the
-            same workload (rank 0, N = 1)
+            the fp64 CPU oracle on the host cores (threads over row blocks),
+            on a bounded sample of the same workload (rank 0, N = 1)
 sweep       per-call microseconds and GB/s of every workload (not timed in
-            the headline number)
+            the headline number); summarised in the JSON line
 """
 from __future__ import annotations
 
@@ -501,12 +504,35 @@ def e2e_measure(ar, device, stream, calls, steps):
     return start.elapsed_time(end) / 1e3, h2d, d2h
 
 
-def oracle_sample(calls, budget_s: float, max_steps: int | None = None, row_fraction: float = 1.0):
+def host_cpu():
+    """Host CPU model and the number of cores this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return {"cpu_model": model, "nproc": n}
+
+
+def oracle_sample(calls, budget_s: float, max_steps: int | None = None, row_fraction: float = 1.0,
+                  threads: int = 1):
     """Time the fp64 CPU oracle (as it stands) on steps of the workload until
     the budget is used or max_steps are done.  A step is every call of the
-    workload, each on its first ceil(row_fraction * T) rows.  Returns
-    (seconds, steps, algorithmic bytes per step actually processed)."""
+    workload, each on its first ceil(row_fraction * T) rows; with threads > 1
+    the rows of each call are split into that many blocks, each computed by
+    one oracle call on its own thread (the oracle's C entry points release
+    the interpreter lock).  Returns (seconds, steps, algorithmic bytes per
+    step actually processed)."""
     import math as _m
+    from concurrent.futures import ThreadPoolExecutor
     import oracle
     from tensor_allreduce_residual_ar_b200 import workloads as wl
     prepared = []
@@ -516,36 +542,54 @@ def oracle_sample(calls, budget_s: float, max_steps: int | None = None, row_frac
         rows = max(1, int(_m.ceil(row_fraction * T)))
         if kind == "qk":
             inp = wl.make_qk_inputs(w, T, dt)
-            prepared.append(("qk", inp, [wl.bits(x)[:rows] for x in inp.qkv]))
+            prepared.append(("qk", inp, rows, [wl.bits(x)[:rows] for x in inp.qkv]))
             step_bytes += wl.qk_bytes(rows, w.W, w.q_size, w.kv_size)
         else:
             inp = wl.make_norm_inputs(w, T, dt)
             res = wl.bits(inp.residual)[:rows] if inp.residual is not None else None
-            prepared.append(("norm", inp, ([wl.bits(p)[:rows] for p in inp.partials], res)))
+            prepared.append(("norm", inp, rows, ([wl.bits(p)[:rows] for p in inp.partials], res)))
             step_bytes += wl.norm_bytes(rows, w.H, w.W, w.residual is not None, w.write_residual,
                                         fp8=w.fp8)
+    fp8 = {id(inp): call[1].fp8 for call, (_, inp, _, _) in zip(calls, prepared)}
+
+    def block(kind, inp, arrs, a, b):
+        if kind == "qk":
+            oracle.qk_norm_sharded([x[a:b] for x in arrs], wl.bits(inp.q_weight),
+                                   wl.bits(inp.k_weight), inp.q_size, inp.kv_size, inp.eps,
+                                   wl.DTYPE_CODE[inp.dtype])
+            return
+        parts, res = arrs
+        o = oracle.ar_add_rmsnorm([p[a:b] for p in parts], None if res is None else res[a:b],
+                                  wl.bits(inp.weight), inp.eps, inp.gemma, wl.DTYPE_CODE[inp.dtype])
+        oracle.round16(o["y"], wl.DTYPE_CODE[inp.dtype])
+        if inp.write_residual:
+            oracle.round16(o["r"], wl.DTYPE_CODE[inp.dtype])
+        if fp8[id(inp)]:
+            oracle.quant_fp8_group(o["y"])
+
+    pool = ThreadPoolExecutor(threads) if threads > 1 else None
 
     def one_step():
-        for kind, inp, arrs in prepared:
-            if kind == "qk":
-                oracle.qk_norm_sharded(arrs, wl.bits(inp.q_weight), wl.bits(inp.k_weight),
-                                       inp.q_size, inp.kv_size, inp.eps, wl.DTYPE_CODE[inp.dtype])
-            else:
-                parts, res = arrs
-                o = oracle.ar_add_rmsnorm(parts, res, wl.bits(inp.weight), inp.eps, inp.gemma,
-                                          wl.DTYPE_CODE[inp.dtype])
-                oracle.round16(o["y"], wl.DTYPE_CODE[inp.dtype])
-                if inp.write_residual:
-                    oracle.round16(o["r"], wl.DTYPE_CODE[inp.dtype])
-    one_step()   # warm (builds the oracle library, page-faults the arrays)
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        one_step()
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or (max_steps is not None and n >= max_steps):
-            break
+        for kind, inp, rows, arrs in prepared:
+            if pool is None:
+                block(kind, inp, arrs, 0, rows)
+                continue
+            n = min(threads, rows)
+            cuts = [rows * i // n for i in range(n + 1)]
+            list(pool.map(lambda i: block(kind, inp, arrs, cuts[i], cuts[i + 1]), range(n)))
+    try:
+        one_step()   # warm (builds the oracle library, page-faults the arrays)
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            one_step()
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s or (max_steps is not None and n >= max_steps):
+                break
+    finally:
+        if pool is not None:
+            pool.shutdown()
     return el, n, step_bytes
 
 
@@ -554,27 +598,31 @@ def oracle_sample(calls, budget_s: float, max_steps: int | None = None, row_frac
 # ----------------------------------------------------------------------------
 
 def run_reference(args):
-    """The reference arm: the fp64 CPU oracle on the host cores, on the same
-    workload, metric and unit; each step a bounded sample of the workload
-    (every call, the first rows of each) so K + W steps take ~2 minutes."""
+    """The reference arm: the fp64 CPU oracle on the host cores (threads over
+    row blocks), on the same workload, metric and unit; each step a bounded
+    sample of the workload (every call, the first rows of each) so K + W
+    steps take about two minutes."""
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
     calls = workload_calls(args.workload)
-    t_full, _, _ = oracle_sample(calls, 0.0, max_steps=1)        # one full step, timed
+    cpu = host_cpu()
+    threads = cpu["nproc"]
+    t_full, _, _ = oracle_sample(calls, 0.0, max_steps=1, threads=threads)   # one full step, timed
     total_budget = 120.0
     frac = min(1.0, total_budget / max(1e-9, t_full * (args.steps + args.warmup)))
-    oracle_sample(calls, 0.0, max_steps=args.warmup, row_fraction=frac)
-    el, n, step_bytes = oracle_sample(calls, float("inf"), max_steps=args.steps, row_fraction=frac)
+    oracle_sample(calls, 0.0, max_steps=args.warmup, row_fraction=frac, threads=threads)
+    el, n, step_bytes = oracle_sample(calls, float("inf"), max_steps=args.steps, row_fraction=frac,
+                                      threads=threads)
     value = step_bytes * n / el / 1e9
     sample = (f"{n} steps of the {args.workload} workload ({len(calls)} calls each, "
-              f"first {frac:.3g} of each call's rows), single-threaded C fp64")
+              f"first {frac:.3g} of each call's rows), C fp64 on {threads} threads")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
             "n_gpus": world, "steps": n, "warmup": args.warmup, "ms_per_step": round(el / n * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": describe(args.workload)},
-            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(value, 5),
-                             "unit": "GB/s"},
+            "cpu_baseline": {"kind": "oracle", "cores": threads, "sample": sample,
+                             "value": round(value, 5), "unit": "GB/s", **cpu},
             "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -659,26 +707,22 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el_max / args.steps * 1e3, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic (seeded torch.randn, distributions of the workload)",
+            "data": "synthetic (seeded torch.randn, the workload's distributions)",
             "config": {"workload": describe(args.workload), "calls_per_step": len(calls),
                        "bytes_per_step": step_bytes, "storage": ",".join(sorted({c[3] for c in calls})),
-                       "l2": (f"{R} rotating buffer sets, a set is reused after "
-                              f">{(R - 1) * step_bytes / 2**20:.0f} MiB of other traffic (L2 126 MiB)"
-                              if R > 1 else "inputs larger than L2"),
-                       "timing": "CUDA graph per buffer set, CUDA events around exactly K steps, "
-                                 "max over ranks",
-                       "parallelism": f"replicas x{world} (independent calls per GPU, no collective)"},
+                       "plans": sorted({plan_of(ar, c) for c in calls}),
+                       "l2": (f"{R} rotating buffer sets, each reused after "
+                              f">{(R - 1) * step_bytes / 2**20:.0f} MiB of other traffic"
+                              if R > 1 else "inputs larger than L2 (126 MiB)"),
+                       "parallelism": f"replicas x{world}, no collective"},
             "us_per_call": round(el_max / args.steps / len(calls) * 1e6, 3),
             "gpu_launches": launches,
             "roofline": {"bound": "hbm", "achieved": round(per_rank_gbs, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(per_rank_gbs / peak, 4),
-                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
-                         if peak_src == "measured" else "fallback 6.65 TB/s",
+                         "peak_source": "measured hbm_gbs" if peak_src == "measured"
+                         else "fallback 6.65 TB/s",
                          "frac_of_8TBps": round(per_rank_gbs / NOMINAL_HBM_GBS, 4),
                          "traffic": ncu_traffic(args.workload),
-                         "traffic_scope": "DRAM read+write bytes per step (all launches of one step), "
-                                          "from one ncu launch list; algorithmic bytes per step in "
-                                          "config.bytes_per_step",
                          "kernel": "norm_rows_kernel" if args.workload != "qk" else "qk_norm_kernel"},
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -694,17 +738,59 @@ def run_ours(args):
     if rank != 0:
         return 0
     if not args.no_sweep:
-        names = ["tiny", "decode", "prefill", "fp8", "qk"] if args.sweep == "all" else \
+        names = ["tiny", "decode", "qk", "fp8", "prefill"] if args.sweep == "all" else \
             [n for n in args.sweep.split(",") if n]
-        line["sweep"] = per_call_sweep(ar, device, stream, names)
+        sweep = per_call_sweep(ar, device, stream, names)
+        for name, rows in sweep.items():
+            for r in rows:
+                hot = f" (hot L2 {r['us_hot_l2']} us)" if "us_hot_l2" in r else ""
+                print(f"sweep {name} T={r['T']} {r['dtype']}: {r['us']} us{hot}, {r['GBps']} GB/s, "
+                      f"{r['frac_of_measured']} of measured, {r['frac_of_8TBps']} of 8 TB/s, "
+                      f"plan {r['plan']}", flush=True)
+        if args.sweep_out:
+            with open(args.sweep_out, "w") as f:
+                json.dump(sweep, f, indent=1)
+        line["sweep_summary"] = sweep_summary(sweep)
     if world == 1 and not args.no_cpu_baseline:
-        el_c, n_c, sb = oracle_sample(calls, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": round(sb * n_c / el_c / 1e9, 5), "unit": "GB/s", "cores": 1,
-                                "kind": "oracle",
-                                "sample": f"{n_c} full steps of the {args.workload} workload "
-                                          f"({len(calls)} calls each) in {el_c:.1f} s, single-threaded C fp64"}
+        cpu = host_cpu()
+        threads = cpu["nproc"]
+        el_c, n_c, sb = oracle_sample(calls, args.cpu_seconds, threads=threads)
+        el_1, n_1, sb_1 = oracle_sample(calls, 0.0, max_steps=1, threads=1,
+                                        row_fraction=min(1.0, 1.0 / max(1, threads)))
+        line["cpu_baseline"] = {
+            "value": round(sb * n_c / el_c / 1e9, 5), "unit": "GB/s", "cores": threads,
+            "kind": "oracle", **cpu,
+            "value_1_thread": round(sb_1 * n_1 / el_1 / 1e9, 5),
+            "sample": f"{n_c} full steps of the {args.workload} workload in {el_c:.1f} s, C fp64 "
+                      f"on {threads} threads over row blocks; value_1_thread: one step on the "
+                      f"first 1/{max(1, threads)} of the rows, one thread"}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def sweep_summary(sweep):
+    """The sweep rows the targets are about, compact: per-call us and the
+    fractions of the measured and the 8 TB/s roofline."""
+    out = {}
+
+    def pick(name, T, dtype="bf16"):
+        for r in sweep.get(name, []):
+            if r["T"] == T and r["dtype"] == dtype:
+                return [r["us"], r["frac_of_measured"], r["frac_of_8TBps"], r["plan"]]
+        return None
+
+    for key, args in (("prefill_T8192", ("prefill", 8192)), ("fp8_T2048", ("fp8", 2048)),
+                      ("fp8_T8192", ("fp8", 8192)), ("fp8_T32768", ("fp8", 32768)),
+                      ("qk_T2048", ("qk", 2048)), ("tiny_T16", ("tiny", 16))):
+        v = pick(*args)
+        if v is not None:
+            out[key] = v
+    dec = sweep.get("decode", [])
+    if dec:
+        out["decode_us_min_max"] = [min(r["us"] for r in dec), max(r["us"] for r in dec)]
+        out["decode_T80_bf16"] = pick("decode", 80)
+    out["fields"] = "us/call, frac of measured peak, frac of 8 TB/s, plan"
+    return out
 
 
 def main(argv=None):
@@ -713,9 +799,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "tiny", "prefill", "fp8", "qk"], default="decode")
+    ap.add_argument("--workload", choices=["prefill", "decode", "tiny", "fp8", "qk"], default="prefill")
     ap.add_argument("--sweep", default="all", help="workloads for the per-call sweep (comma list or all)")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--sweep-out", default=None, help="also write the full sweep as JSON here")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--spin-seconds", type=float, default=0.5,

@@ -210,16 +210,23 @@ typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_v
  *   ROWC<k>           one row per cluster of k CTAs; the sum of squares is
  *                     combined through distributed shared memory.
  *   PERSIST           one CTA of at most 256 threads per row; persistent grid
- *                     (SM count x occupancy), rows looped, each CTA's next
- *                     row bulk-prefetched into L2.
- *   PERSIST512        the same with at most 512 threads, two CTAs per SM.
- *   PERSIST_C2        the same with each row split over a cluster of 2 CTAs;
- *                     the grid is the number of clusters that fit at once.
- *   PERSIST_AHEAD     one CTA of at most 512 threads per row, persistent; each
- *                     thread's next row is loaded into registers while the
- *                     current one is finished (where the register budget
- *                     allows).
- *   PERSIST_C2_AHEAD  the same with each row split over a cluster of 2 CTAs.
+ *                     (SM count x occupancy), rows looped.  Where a thread's
+ *                     share of a row fits the register budget (at most 10
+ *                     16-byte packs: packs per thread x (W + 1)) the CTA's
+ *                     next row is loaded into registers while the current
+ *                     one is finished; otherwise it is bulk-prefetched into
+ *                     L2.
+ *   PERSIST_AHEAD     the same with at most 512 threads (fewer packs per
+ *                     thread, so the register load-ahead applies to wider
+ *                     rows).
+ *   PERSIST_C2_AHEAD  PERSIST_AHEAD with each row split over a cluster of 2
+ *                     CTAs; the grid is the number of clusters that fit at
+ *                     once.
+ *   PERSIST512        persistent, at most 512 threads, two CTAs per SM
+ *                     (registers for two CTAs, so no load-ahead); each CTA's
+ *                     next row is bulk-prefetched into L2.
+ *   PERSIST_C2        PERSIST512 with each row split over a cluster of 2
+ *                     CTAs.
  *   BULK              rows staged into shared memory by bulk asynchronous
  *                     copies.
  *   QK_C<k>           one token per cluster of k CTAs, shards split across

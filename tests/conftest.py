@@ -35,6 +35,25 @@ def lib(cuda_device):
     return ar
 
 
+@pytest.fixture(scope="session")
+def parity_report():
+    """Collects per-workload error statistics from the GPU parity tests.
+    When AR_PARITY_REPORT names a file, the collected lines are written there
+    as JSON at the end of the session (nothing is written otherwise)."""
+    import json
+    rows = []
+
+    def add(name, stats):
+        rows.append({"case": name, **{k: v for k, v in stats.items()}})
+
+    yield add
+    path = os.environ.get("AR_PARITY_REPORT")
+    if path and rows:
+        with open(path, "w") as f:
+            for r in rows:
+                f.write(json.dumps(r) + "\n")
+
+
 @pytest.fixture(autouse=True)
 def _clear_forced_plans(request):
     """A plan forced by one test never leaks into the next: after every test

@@ -2,9 +2,12 @@
 that run one workload instance through both.
 
 Tolerances:
-  * 16-bit y: per element |g - o| <= 4e-3 |o|, or g within one unit in the
-    last place of RNE(o) (covers exact zeros and fp16 subnormals where
-    rounding alone exceeds 4e-3);
+  * 16-bit y: per element |g - o| <= 4e-3 |o|.  Only where o is zero or
+    below the format's smallest normal number (fp16 subnormals, where the
+    fixed spacing makes rounding alone exceed 4e-3 relative) may g instead be
+    within one unit in the last place of RNE(o).  For normal outputs RNE
+    itself is within half a unit, 2^-8 < 4e-3 relative in bf16 and 2^-11 in
+    fp16, so the relative bound is the whole test there;
   * residual_out: within one ulp of RNE(r), r the exact fp64 sum;
   * FP8 codes: within one e4m3 step (adjacent codes in value order);
   * FP8 scales: within 1e-6 relative of amax/448 in fp64.
@@ -19,6 +22,8 @@ from tensor_allreduce_residual_ar_b200 import workloads as wl
 
 Y_RTOL = 4e-3
 SCALE_RTOL = 1e-6
+# smallest positive normal number of each 16-bit format
+MIN_NORMAL = {"bf16": 2.0 ** -126, "fp16": 2.0 ** -14}
 
 
 def ordinal16(bits: np.ndarray) -> np.ndarray:
@@ -33,10 +38,16 @@ def ordinal8(codes: np.ndarray) -> np.ndarray:
 
 
 def check_y(gpu_bits: np.ndarray, y64: np.ndarray, dtype: str, what: str = "y"):
+    """Per-element check of 16-bit outputs against the fp64 oracle.  Returns
+    the largest and the 99.99th-percentile relative error over non-zero
+    oracle values, the number of elements that needed the one-ulp clause
+    (all of them zero or subnormal in the output format), and how many
+    elements lay in that range at all."""
     dt = wl.DTYPE_CODE[dtype]
     g = oracle.decode16(gpu_bits, dt)
     rel_ok = np.abs(g - y64) <= Y_RTOL * np.abs(y64)
-    ulp_ok = np.abs(ordinal16(gpu_bits) - ordinal16(oracle.round16(y64, dt))) <= 1
+    tiny = np.abs(y64) < MIN_NORMAL[dtype]
+    ulp_ok = tiny & (np.abs(ordinal16(gpu_bits) - ordinal16(oracle.round16(y64, dt))) <= 1)
     bad = ~(rel_ok | ulp_ok)
     nbad = int(bad.sum())
     if nbad:
@@ -45,8 +56,13 @@ def check_y(gpu_bits: np.ndarray, y64: np.ndarray, dtype: str, what: str = "y"):
                              f"gpu {g[bad][:5]} oracle {y64[bad][:5]}")
     nz = y64 != 0
     rel = np.abs(g[nz] - y64[nz]) / np.abs(y64[nz])
+    normal = ~tiny
+    rel_n = np.abs(g[normal] - y64[normal]) / np.abs(y64[normal])
     return {"max_rel": float(rel.max()) if rel.size else 0.0,
-            "ulp_clause": int((~rel_ok & ulp_ok).sum())}
+            "max_rel_normal": float(rel_n.max()) if rel_n.size else 0.0,
+            "p9999_rel": float(np.quantile(rel, 0.9999)) if rel.size else 0.0,
+            "ulp_clause": int((~rel_ok & ulp_ok).sum()),
+            "tiny": int(tiny.sum())}
 
 
 def check_res(gpu_bits: np.ndarray, r64: np.ndarray, dtype: str):

@@ -45,3 +45,41 @@ def test_e2e_staging_views_alias_one_slab():
         assert dout.data_ptr() <= t.data_ptr() < dout.data_ptr() + out_pad
     assert in_bytes == sum(t.numel() * t.element_size() for t in b.inputs())
     assert out_bytes == sum(t.numel() * t.element_size() for t in b.outputs())
+
+
+def test_oracle_sample_threads_cover_every_row():
+    """Threaded oracle timing splits each call's rows into blocks; the bytes
+    counted are those of the whole sample either way."""
+    calls = bench.workload_calls("tiny")
+    _, n1, b1 = bench.oracle_sample(calls, 0.0, max_steps=1, threads=1)
+    _, n3, b3 = bench.oracle_sample(calls, 0.0, max_steps=1, threads=3)
+    assert n1 == n3 == 1 and b1 == b3 == bench.call_bytes(calls[0])
+    cpu = bench.host_cpu()
+    assert cpu["nproc"] >= 1
+
+
+def test_oracle_rows_are_independent():
+    """What threading over row blocks relies on: the oracle's rows do not
+    depend on each other, so blocks computed separately equal the whole."""
+    import numpy as np
+    import oracle
+    from tensor_allreduce_residual_ar_b200 import workloads as wl
+    inp = wl.make_norm_inputs(wl.TINY, 16, H=256)
+    parts = [wl.bits(p) for p in inp.partials]
+    res = wl.bits(inp.residual)
+    whole = oracle.ar_add_rmsnorm(parts, res, wl.bits(inp.weight), inp.eps, False, 0)["y"]
+    blocks = [oracle.ar_add_rmsnorm([p[a:b] for p in parts], res[a:b], wl.bits(inp.weight),
+                                    inp.eps, False, 0)["y"] for a, b in ((0, 5), (5, 11), (11, 16))]
+    assert np.array_equal(whole, np.concatenate(blocks))
+
+
+def test_sweep_summary_fields():
+    sweep = {"prefill": [{"T": 8192, "dtype": "bf16", "us": 104.0, "frac_of_measured": 0.98,
+                          "frac_of_8TBps": 0.8, "plan": 9}],
+             "decode": [{"T": 1, "dtype": "bf16", "us": 2.5, "frac_of_measured": 0.01,
+                         "frac_of_8TBps": 0.01, "plan": 4},
+                        {"T": 80, "dtype": "bf16", "us": 4.2, "frac_of_measured": 0.3,
+                         "frac_of_8TBps": 0.27, "plan": 4}]}
+    s = bench.sweep_summary(sweep)
+    assert s["prefill_T8192"] == [104.0, 0.98, 0.8, 9]
+    assert s["decode_us_min_max"] == [2.5, 4.2] and s["decode_T80_bf16"][0] == 4.2

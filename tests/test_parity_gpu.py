@@ -89,23 +89,33 @@ def check_norm(lib, inp, **kw):
 # the five workloads
 # ----------------------------------------------------------------------------
 
-def test_tiny(lib):
-    check_norm(lib, wl.make_norm_inputs(wl.TINY, 16))
+def test_tiny(lib, parity_report):
+    st = check_norm(lib, wl.make_norm_inputs(wl.TINY, 16))
+    assert st["ulp_clause"] == 0
+    parity_report("tiny T=16 y", st)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("T", wl.DECODE.Ts)
-def test_decode_window(lib, T, dtype):
-    check_norm(lib, wl.make_norm_inputs(wl.DECODE, T, dtype))
+def test_decode_window(lib, T, dtype, parity_report):
+    st = check_norm(lib, wl.make_norm_inputs(wl.DECODE, T, dtype))
+    if dtype == "bf16":
+        assert st["ulp_clause"] == 0
+    parity_report(f"decode T={T} {dtype} y", st)
 
 
-def test_prefill_dead_residual_full(lib):
+def test_prefill_dead_residual_full(lib, parity_report):
     inp = wl.make_norm_inputs(wl.PREFILL, 8192)
     assert not inp.write_residual
-    check_norm(lib, inp)
+    st = check_norm(lib, inp)
+    assert st["ulp_clause"] == 0
+    parity_report("prefill T=8192 y", st)
 
 
 def run_fp8(lib, inp, *, with_y=True, with_res=True, plan=None):
+    """One FP8-variant call on guarded buffers.  With inp.residual None it is
+    the no-residual form (r is the plain sum of the partials); residual_out
+    is still written when with_res is set."""
     dev = "cuda"
     T, H = inp.T, inp.H
     parts = [p.to(dev) for p in inp.partials]
@@ -136,25 +146,44 @@ def check_fp8(lib, inp, rows=None, **kw):
         r = r[rows] if r is not None else None
     st = P.check_fp8(q, s, o["y"])
     if y is not None:
-        P.check_y(y, o["y"], inp.dtype)
+        sy = P.check_y(y, o["y"], inp.dtype)
+        if inp.dtype == "bf16":
+            assert sy["ulp_clause"] == 0
+        st.update({"y_" + k: v for k, v in sy.items()})
     if r is not None:
         P.check_res(r, o["r"], inp.dtype)
     return st
 
 
 @pytest.mark.parametrize("T", wl.FP8.Ts)
-def test_fp8_group_sweep(lib, T):
+def test_fp8_group_sweep(lib, T, parity_report):
     inp = wl.make_norm_inputs(wl.FP8, T)
     rows = None
     if T > 2048:   # sampled rows at the largest sizes: first, last and 62 spread
         rng = np.random.default_rng(T)
         rows = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 62, replace=False)]))
-    check_fp8(lib, inp, rows=rows)
+    st = check_fp8(lib, inp, rows=rows)
+    parity_report(f"fp8 T={T} codes/scales", st)
+
+
+@pytest.mark.parametrize("plan", NORM_PLANS)
+def test_fp8_no_residual_every_plan(lib, plan):
+    """The no-residual FP8 site (all_reduce -> rms_norm -> per-group quant):
+    residual NULL, so r is the plain sum of the partials.  Codes, scales,
+    the 16-bit y and residual_out (the sum itself) against the oracle, on
+    row, persistent and bulk-staged plans, ragged shapes included."""
+    for T, H, W in ((1, 128, 1), (7, 640, 3), (67, 5120, 4), (300, 2048, 8)):
+        inp = wl.make_norm_inputs(wl.FP8, T, W=W, H=H, residual=False, seed=3000 + T + H + W)
+        assert inp.residual is None
+        st = check_fp8(lib, inp, plan=plan)
+        assert st["scale_max_rel"] <= P.SCALE_RTOL
 
 
 @pytest.mark.parametrize("T", wl.QK.Ts)
-def test_qk_sharded(lib, T):
-    check_qk(lib, wl.make_qk_inputs(wl.QK, T))
+def test_qk_sharded(lib, T, parity_report):
+    st = check_qk(lib, wl.make_qk_inputs(wl.QK, T))
+    assert st["ulp_clause"] == 0
+    parity_report(f"qk T={T} q,k", st)
 
 
 def run_qk(lib, inp, plan=None):
@@ -177,11 +206,18 @@ def run_qk(lib, inp, plan=None):
 
 
 def check_qk(lib, inp, plan=None):
+    """Every shard's q and k outputs against the oracle; returns the worst
+    statistics over all of them."""
     qo, ko = run_qk(lib, inp, plan)
     q64, k64 = P.oracle_qk(inp)
+    worst = {"max_rel": 0.0, "p9999_rel": 0.0, "ulp_clause": 0}
     for w in range(inp.W):
-        P.check_y(qo[w], q64[w], inp.dtype, f"q_out[{w}]")
-        P.check_y(ko[w], k64[w], inp.dtype, f"k_out[{w}]")
+        for st in (P.check_y(qo[w], q64[w], inp.dtype, f"q_out[{w}]"),
+                   P.check_y(ko[w], k64[w], inp.dtype, f"k_out[{w}]")):
+            worst["max_rel"] = max(worst["max_rel"], st["max_rel"])
+            worst["p9999_rel"] = max(worst["p9999_rel"], st["p9999_rel"])
+            worst["ulp_clause"] += st["ulp_clause"]
+    return worst
 
 
 # ----------------------------------------------------------------------------
