@@ -48,17 +48,35 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    """Compile every source to an object file (in parallel, one nvcc per
+    translation unit), then link the shared library."""
     if not force and up_to_date():
         return OUT
     os.makedirs(os.path.dirname(OUT), exist_ok=True)
-    tmp = OUT + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC,
-           "--expt-relaxed-constexpr", "-DAR_BUILDING_LIBRARY", "-o", tmp, *sources()]
+    objdir = os.path.join(os.path.dirname(OUT), f"obj{os.getpid()}")
+    os.makedirs(objdir, exist_ok=True)
+    common = [_nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
+              "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC,
+              "--expt-relaxed-constexpr", "-DAR_BUILDING_LIBRARY"]
     if ptxas_verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, OUT)
+        common.insert(1, "-Xptxas=-v")
+    procs, objs = [], []
+    try:
+        for src in sources():
+            obj = os.path.join(objdir, os.path.basename(src) + ".o")
+            objs.append(obj)
+            procs.append((src, subprocess.Popen([*common, "-c", "-o", obj, src])))
+        failed = [src for src, pr in procs if pr.wait() != 0]
+        if failed:
+            raise subprocess.CalledProcessError(1, f"nvcc {' '.join(failed)}")
+        tmp = OUT + f".tmp{os.getpid()}"
+        subprocess.run([_nvcc(), *ARCH, "-shared", "-o", tmp, *objs], check=True)
+        os.replace(tmp, OUT)
+    finally:
+        for _, pr in procs:
+            if pr.poll() is None:
+                pr.kill()
+        shutil.rmtree(objdir, ignore_errors=True)
     return OUT
 
 

@@ -13,20 +13,15 @@
 #include <mutex>
 
 #include "ar_rmsnorm.h"
+#include "host_util.h"
 #include "kernels.cuh"
 #include "plan.h"
 
 using namespace arn;
 
-namespace {
+namespace arn {
 
 constexpr int kMaxDevices = 64;
-
-struct DevInfo {
-    int sm_count = 0;
-    int smem_optin = 0;   // largest dynamic shared memory per block
-    int status = AR_OK;
-};
 
 DevInfo g_dev[kMaxDevices];
 std::once_flag g_dev_once[kMaxDevices];
@@ -54,11 +49,86 @@ int device_info(DevInfo &out) {
     return out.status;
 }
 
+bool split_threads(int packs, int max_threads, int &threads, int &ppt_idx) {
+    for (int i = 0; i < kPptVariants; ++i) {
+        const int ppt = 1 << i;
+        const int t = (packs + ppt - 1) / ppt;
+        if (t <= max_threads) {
+            threads = ((t + 31) / 32) * 32;
+            ppt_idx = i;
+            return true;
+        }
+    }
+    return false;
+}
+
+namespace {
+struct OccKey { const void *fn; int threads; int dev; };
+struct OccSlot { OccKey key; int occ; };
+std::mutex g_occ_mutex;
+OccSlot g_occ[512];
+int g_occ_n = 0;
+struct ClusterOccSlot { OccKey key; int C; int n; };
+ClusterOccSlot g_cocc[256];
+int g_cocc_n = 0;
+}  // namespace
+
+int occupancy(const void *fn, int threads, int dev) {
+    std::lock_guard<std::mutex> lk(g_occ_mutex);
+    for (int i = 0; i < g_occ_n; ++i)
+        if (g_occ[i].key.fn == fn && g_occ[i].key.threads == threads && g_occ[i].key.dev == dev)
+            return g_occ[i].occ;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, 0) != cudaSuccess || occ < 1)
+        occ = 1;
+    if (g_occ_n < 512) g_occ[g_occ_n++] = {{fn, threads, dev}, occ};
+    return occ;
+}
+
+int cluster_occupancy(const void *fn, int threads, int C, int dev, int sm_count) {
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mutex);
+        for (int i = 0; i < g_cocc_n; ++i)
+            if (g_cocc[i].key.fn == fn && g_cocc[i].key.threads == threads &&
+                g_cocc[i].key.dev == dev && g_cocc[i].C == C)
+                return g_cocc[i].n;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)C, 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = (unsigned)C;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        n = sm_count * occupancy(fn, threads, dev) / C;
+    }
+    if (n < 1) n = 1;
+    std::lock_guard<std::mutex> lk(g_occ_mutex);
+    if (g_cocc_n < 256) g_cocc[g_cocc_n++] = {{fn, threads, dev}, C, n};
+    return n;
+}
+
+// Programmatic dependent launch is on unless AR_RMSNORM_PDL=0 in the
+// environment when the library first launches.
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("AR_RMSNORM_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+}  // namespace arn
+
+namespace {
+
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
-constexpr int kPptVariants = 3;   // packs per thread 1, 2, 4
-
-int wb_bucket(int W) { return W <= 2 ? 0 : W <= 4 ? 1 : W <= 8 ? 2 : 3; }   // 2, 4, 8, 16
 
 // ---------------------------------------------------------------------------
 // launch tables
@@ -155,50 +225,6 @@ QKKernel pick_qk_kernel(int dtype, int ppt_idx, int minb) {
     return dtype == AR_BF16 ? bf[m][ppt_idx] : hf[m][ppt_idx];
 }
 
-// Threads per CTA and packs per thread for `packs` packs per CTA: the
-// fewest packs per thread (1, 2, 4) that fit within max_threads.
-bool split_threads(int packs, int max_threads, int &threads, int &ppt_idx) {
-    for (int i = 0; i < kPptVariants; ++i) {
-        const int ppt = 1 << i;
-        const int t = (packs + ppt - 1) / ppt;
-        if (t <= max_threads) {
-            threads = ((t + 31) / 32) * 32;
-            ppt_idx = i;
-            return true;
-        }
-    }
-    return false;
-}
-
-// Occupancy (resident CTAs per SM) of a kernel at a block size, cached.
-struct OccKey { const void *fn; int threads; int dev; };
-struct OccSlot { OccKey key; int occ; };
-std::mutex g_occ_mutex;
-OccSlot g_occ[256];
-int g_occ_n = 0;
-
-int occupancy(const void *fn, int threads, int dev) {
-    std::lock_guard<std::mutex> lk(g_occ_mutex);
-    for (int i = 0; i < g_occ_n; ++i)
-        if (g_occ[i].key.fn == fn && g_occ[i].key.threads == threads && g_occ[i].key.dev == dev)
-            return g_occ[i].occ;
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, 0) != cudaSuccess || occ < 1)
-        occ = 1;
-    if (g_occ_n < 256) g_occ[g_occ_n++] = {{fn, threads, dev}, occ};
-    return occ;
-}
-
-// Programmatic dependent launch is on unless AR_RMSNORM_PDL=0 in the
-// environment when the library first launches.
-bool pdl_enabled() {
-    static const bool on = [] {
-        const char *e = std::getenv("AR_RMSNORM_PDL");
-        return !(e && e[0] == '0');
-    }();
-    return on;
-}
-
 template <typename Params>
 int launch(void (*fn)(const Params), const Params &p, int64_t clusters, int C, int threads,
            cudaStream_t stream, size_t smem = 0) {
@@ -226,41 +252,6 @@ int launch(void (*fn)(const Params), const Params &p, int64_t clusters, int C, i
     cfg.attrs = na ? attr : nullptr;
     cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, fn, p) == cudaSuccess ? AR_OK : AR_ECUDA;
-}
-
-// Clusters of C CTAs of a kernel that can be resident at once on the whole
-// device (cluster placement within GPCs included), cached.
-struct ClusterOccSlot { OccKey key; int C; int n; };
-ClusterOccSlot g_cocc[64];
-int g_cocc_n = 0;
-
-int cluster_occupancy(const void *fn, int threads, int C, int dev, int sm_count) {
-    {
-        std::lock_guard<std::mutex> lk(g_occ_mutex);
-        for (int i = 0; i < g_cocc_n; ++i)
-            if (g_cocc[i].key.fn == fn && g_cocc[i].key.threads == threads &&
-                g_cocc[i].key.dev == dev && g_cocc[i].C == C)
-                return g_cocc[i].n;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)C, 1, 1);
-    cfg.blockDim = dim3((unsigned)threads, 1, 1);
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = (unsigned)C;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
-        (void)cudaGetLastError();
-        n = sm_count * occupancy(fn, threads, dev) / C;
-    }
-    if (n < 1) n = 1;
-    std::lock_guard<std::mutex> lk(g_occ_mutex);
-    if (g_cocc_n < 64) g_cocc[g_cocc_n++] = {{fn, threads, dev}, C, n};
-    return n;
 }
 
 // Grid size in clusters: one per row, or capped for persistent plans.
