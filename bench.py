@@ -594,6 +594,116 @@ def oracle_sample(calls, budget_s: float, max_steps: int | None = None, row_frac
 
 
 # ----------------------------------------------------------------------------
+# multi-GPU form (N > 1): the fused exchange kernels against NCCL
+# ----------------------------------------------------------------------------
+
+TP_SHAPES = ((1, 8192), (8, 8192), (32, 8192), (80, 8192), (256, 8192), (1024, 8192), (8192, 4096))
+TP_QK_TS = (1, 64, 2048)
+
+
+def tp_crossover(rows):
+    """From [T, H, one-shot us, two-shot us, NCCL us] rows: the first T where
+    two-shot beats one-shot, and the first where the better fused form loses
+    to NCCL all-reduce + norm (None when it never happens)."""
+    two_wins = next((r[0] for r in rows if r[2] is not None and r[3] is not None and r[3] < r[2]), None)
+    nccl_wins = next((r[0] for r in rows
+                      if r[4] is not None and min(x for x in (r[2], r[3]) if x is not None) > r[4]), None)
+    return {"twoshot_beats_oneshot_from_T": two_wins, "nccl_beats_fused_from_T": nccl_wins}
+
+
+def tp_arm(ar, device, stream, world, rank, iters=100):
+    """Per shape: the fused one-shot and two-shot pull kernels, and the
+    unfused baseline (copy of the partial, NCCL all_reduce, then this
+    library's add + RMSNorm with W = 1), each timed over `iters` calls with
+    CUDA events on the launching stream, max over ranks.  Every rank takes the
+    same steps in the same order."""
+    import torch
+    import torch.distributed as dist
+    from tensor_allreduce_residual_ar_b200 import comm as C
+    comm = C.Comm(8192 * 8192, device=device)
+    rows, worst = [], 0.0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(10):
+            fn()
+        torch.cuda.synchronize()
+        barrier(device)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(iters):
+                fn()
+            ev1.record(stream)
+        ev1.synchronize()
+        return max_over_ranks(ev0.elapsed_time(ev1) / iters * 1e3, device)
+
+    try:
+        for T, H in TP_SHAPES:
+            g = torch.Generator(device=device).manual_seed(7000 + T)          # same on every rank
+            res = torch.randn(T, H, generator=g, device=device).to(torch.bfloat16)
+            w = (1 + 0.1 * torch.randn(H, generator=g, device=device)).to(torch.bfloat16)
+            gp = torch.Generator(device=device).manual_seed(8000 + 131 * rank + T)
+            part = (0.5 * torch.randn(T, H, generator=gp, device=device)).to(torch.bfloat16)
+            out, rout = torch.empty_like(part), torch.empty_like(part)
+            buf, ref, rref = torch.empty_like(part), torch.empty_like(part), torch.empty_like(part)
+
+            def baseline():
+                with torch.cuda.stream(stream):
+                    buf.copy_(part)
+                    dist.all_reduce(buf)
+                    ar.ar_add_rmsnorm([buf], res, w, ref, rref, eps=1e-6)
+
+            def fused(algo):
+                return lambda: comm.allreduce_add_rmsnorm(part, res, w, out, rout, eps=1e-6, algo=algo,
+                                                          stream=stream)
+            us = {"nccl": timed(baseline)}
+            for algo in ("oneshot", "twoshot"):
+                if algo == "oneshot" and T * H * 2 > (8 << 20):
+                    us[algo] = None
+                    continue
+                us[algo] = timed(fused(algo))
+                torch.cuda.synchronize()
+                d = ((out.float() - ref.float()).abs() / ref.float().abs().clamp_min(1e-2)).max().item()
+                worst = max(worst, d)
+            rows.append([T, H, None if us["oneshot"] is None else round(us["oneshot"], 2),
+                         round(us["twoshot"], 2), round(us["nccl"], 2)])
+            del part, res, w, out, rout, buf, ref, rref
+        qk = []
+        q_size, kv_size = 6144, 1024
+        qs, ks = q_size // world, kv_size // world
+        for T in TP_QK_TS:
+            g = torch.Generator(device=device).manual_seed(9000 + T)
+            qw = (1 + 0.1 * torch.randn(q_size, generator=g, device=device)).to(torch.bfloat16)
+            kw = (1 + 0.1 * torch.randn(kv_size, generator=g, device=device)).to(torch.bfloat16)
+            gp = torch.Generator(device=device).manual_seed(9500 + 131 * rank + T)
+            qkv = torch.randn(T, qs + 2 * ks, generator=gp, device=device).to(torch.bfloat16)
+            qo, ko = torch.empty((T, qs), dtype=torch.bfloat16, device=device), \
+                torch.empty((T, ks), dtype=torch.bfloat16, device=device)
+
+            def qk_baseline():
+                # the unfused form: sums of squares, NCCL all_reduce, normalise
+                with torch.cuda.stream(stream):
+                    x = qkv.float()
+                    ss = torch.stack([x[:, :qs].pow(2).sum(-1), x[:, qs:qs + ks].pow(2).sum(-1)], -1)
+                    dist.all_reduce(ss)
+                    qo.copy_(x[:, :qs] * torch.rsqrt(ss[:, :1] / q_size + 1e-6) * qw[rank * qs:(rank + 1) * qs])
+                    ko.copy_(x[:, qs:qs + ks] * torch.rsqrt(ss[:, 1:] / kv_size + 1e-6) *
+                             kw[rank * ks:(rank + 1) * ks])
+            t_base = timed(qk_baseline)
+            t_fused = timed(lambda: comm.qk_norm_sharded(qkv, qw, kw, qo, ko, q_size, kv_size, eps=1e-6,
+                                                         stream=stream))
+            qk.append([T, round(t_fused, 2), round(t_base, 2)])
+        status = comm.status()
+    finally:
+        comm.close()
+    return {"norm_us": rows, "norm_fields": "T, H, one-shot, two-shot, copy + NCCL all_reduce + W=1 "
+                                            "norm (us per call, max over ranks; bf16, one partial per rank)",
+            **tp_crossover(rows), "max_rel_vs_nccl_path": round(worst, 5),
+            "qk_us": qk, "qk_fields": "T, fused, torch sums + NCCL all_reduce + normalise",
+            "status": status}
+
+
+# ----------------------------------------------------------------------------
 # arms
 # ----------------------------------------------------------------------------
 
@@ -729,6 +839,12 @@ def run_ours(args):
             "clocks": sampler.summary()}
 
     del graphs
+    if world > 1 and not args.no_tp:
+        # the multi-GPU form itself: fused exchange kernels against NCCL
+        try:
+            line["tp"] = tp_arm(ar, device, stream, world, rank)
+        except Exception as e:            # reported, never hidden
+            line["tp"] = {"error": f"{type(e).__name__}: {str(e)[:300]}"}
     # Every collective is done: the ranks part here, so that rank 0's
     # sweep and oracle timing below (no collectives, a minute or more) keep
     # no other rank waiting in a barrier against the group's timeout.
@@ -804,6 +920,7 @@ def main(argv=None):
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-out", default=None, help="also write the full sweep as JSON here")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tp", action="store_true", help="N > 1: skip the multi-GPU exchange arm")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--spin-seconds", type=float, default=0.5,
                     help="untimed load before the timed region (clocks settle, sampler runs)")

@@ -83,3 +83,12 @@ def test_sweep_summary_fields():
     s = bench.sweep_summary(sweep)
     assert s["prefill_T8192"] == [104.0, 0.98, 0.8, 9]
     assert s["decode_us_min_max"] == [2.5, 4.2] and s["decode_T80_bf16"][0] == 4.2
+
+
+def test_tp_crossover():
+    rows = [[1, 8192, 5.0, 7.0, 12.0], [80, 8192, 8.0, 9.0, 14.0], [256, 8192, 20.0, 15.0, 18.0],
+            [8192, 4096, None, 300.0, 280.0]]
+    c = bench.tp_crossover(rows)
+    assert c == {"twoshot_beats_oneshot_from_T": 256, "nccl_beats_fused_from_T": 8192}
+    assert bench.tp_crossover(rows[:2]) == {"twoshot_beats_oneshot_from_T": None,
+                                            "nccl_beats_fused_from_T": None}
