@@ -234,7 +234,13 @@ typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_v
  *   QK_PERSIST        one CTA of at most 512 threads per token, persistent
  *                     grid with L2 prefetch.
  *   QK_PERSIST256     the same with at most 256 threads (more packs per
- *                     thread). */
+ *                     thread).
+ *   QK_BULK           one persistent CTA per SM; one thread keeps up to 16
+ *                     tokens in flight into a shared-memory ring with bulk
+ *                     asynchronous copies (one per shard row), and whole
+ *                     warps normalise one token each from it (falls back to
+ *                     QK_PERSIST where two tokens and the weights do not fit
+ *                     in shared memory). */
 enum {
     AR_PLAN_AUTO = 0,
     AR_PLAN_ROWC1 = 1,
@@ -252,7 +258,8 @@ enum {
     AR_PLAN_QK_C4 = 13,
     AR_PLAN_QK_C8 = 14,
     AR_PLAN_QK_PERSIST = 15,
-    AR_PLAN_QK_PERSIST256 = 16
+    AR_PLAN_QK_PERSIST256 = 16,
+    AR_PLAN_QK_BULK = 17
 };
 
 /* The plan a call with these arguments would use (for QK, H = q_size + kv_size

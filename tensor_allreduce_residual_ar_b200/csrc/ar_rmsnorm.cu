@@ -482,7 +482,27 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
     p.inv_k = (float)(1.0 / (double)kv_size);
     p.eps = eps;
 
-    const int plan = plan_lookup(AR_VARIANT_QK, T, q_size + kv_size, W, dtype, di.sm_count);
+    int plan = plan_lookup(AR_VARIANT_QK, T, q_size + kv_size, W, dtype, di.sm_count);
+    if (plan == AR_PLAN_QK_BULK) {
+        // weights plus at least two tokens in the shared-memory ring, else
+        // the persistent register-resident plan
+        const size_t tok_bytes = (size_t)W * (size_t)(qs + ks) * 2;
+        const size_t w_bytes = (size_t)(q_size + kv_size) * 2;
+        const size_t budget = (size_t)di.smem_optin > 4096 ? (size_t)di.smem_optin - 4096 : 0;
+        int stages = budget > w_bytes ? (int)((budget - w_bytes) / tok_bytes) : 0;
+        if (stages > kQKMaxStages) stages = kQKMaxStages;
+        if (stages >= 2) {
+            p.C = 1;
+            p.stages = stages;
+            QKKernel fn = dtype == AR_BF16 ? &qk_bulk_kernel<__nv_bfloat16> : &qk_bulk_kernel<__half>;
+            const int smem = (int)(w_bytes + (size_t)stages * tok_bytes);
+            int st2 = ensure_smem((const void *)fn, dev, smem);
+            if (st2 != AR_OK) return st2;
+            const int64_t grid = T < di.sm_count ? T : di.sm_count;
+            return launch(fn, p, grid, 1, kMaxThreads, stream, (size_t)smem);
+        }
+        plan = AR_PLAN_QK_PERSIST;
+    }
     Geometry g = plan_geometry(plan);
     while (g.C > 1 && W % g.C != 0) g.C /= 2;
     int threads = 0, ppt_idx = 0;
