@@ -489,17 +489,20 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
         const size_t tok_bytes = (size_t)W * (size_t)(qs + ks) * 2;
         const size_t w_bytes = (size_t)(q_size + kv_size) * 2;
         const size_t budget = (size_t)di.smem_optin > 4096 ? (size_t)di.smem_optin - 4096 : 0;
-        int stages = budget > w_bytes ? (int)((budget - w_bytes) / tok_bytes) : 0;
-        if (stages > kQKMaxStages) stages = kQKMaxStages;
-        if (stages >= 2) {
+        int fit = budget > w_bytes ? (int)((budget - w_bytes) / tok_bytes) : 0;
+        if (fit > kQKMaxStages) fit = kQKMaxStages;
+        if (fit >= 4) {
+            // NW consumer warps with SPW stages each (stages = NW * SPW)
+            const int nw = fit < kMaxWarps - 1 ? fit : kMaxWarps - 1;
+            const int spw = fit / nw;
             p.C = 1;
-            p.stages = stages;
+            p.stages = nw * spw;
             QKKernel fn = dtype == AR_BF16 ? &qk_bulk_kernel<__nv_bfloat16> : &qk_bulk_kernel<__half>;
-            const int smem = (int)(w_bytes + (size_t)stages * tok_bytes);
+            const int smem = (int)(w_bytes + (size_t)p.stages * tok_bytes);
             int st2 = ensure_smem((const void *)fn, dev, smem);
             if (st2 != AR_OK) return st2;
             const int64_t grid = T < di.sm_count ? T : di.sm_count;
-            return launch(fn, p, grid, 1, kMaxThreads, stream, (size_t)smem);
+            return launch(fn, p, grid, 1, 32 * (nw + 1), stream, (size_t)smem);
         }
         plan = AR_PLAN_QK_PERSIST;
     }
