@@ -194,6 +194,37 @@ AR_API int ar_group_qk_norm_sharded(ar_comm *g, const void *const *qkv, const vo
                                     int64_t T, int64_t q_size, int64_t kv_size, float eps,
                                     int dtype, cudaStream_t stream);
 
+/*
+ * ar_group_qk_norm_sharded_static -- ar_group_qk_norm_sharded (W ranks of
+ * one GPU, one cooperative launch) for callers that cannot allocate device
+ * memory: it calls no cudaMalloc, cudaFree or allocating library routine.
+ * Some callers cannot call cudaMalloc: a plugin that only receives buffers
+ * from its host application, an engine that reserved all free device
+ * memory at start-up (a further allocation would fail), or code that must
+ * not take the device-wide synchronisation cudaMalloc may imply.  The
+ * papers describe no such form: it has no counterpart there.
+ *
+ * The exchange regions live in one file-scope device array of
+ * AR_STATIC_QK_MAX_W regions of 8 * AR_STATIC_QK_MAX_T * 2 bytes plus the
+ * flag area (about 2 MiB), which every GPU that loads the library holds
+ * until the process exits.  The first call on a device looks up the array's
+ * device address on that device (once); make that first call before any
+ * stream capture.  Every call shares the array: each call first clears the
+ * flags and counters of the regions it uses (an asynchronous memset on
+ * `stream`), so calls in one stream are ordered, and calls that overlap on
+ * the GPU (other streams, other threads) race and give undefined results.
+ * 1 <= W <= AR_STATIC_QK_MAX_W and T <= AR_STATIC_QK_MAX_T (else AR_EINVAL /
+ * AR_EUNSUPPORTED); other arguments as in ar_group_qk_norm_sharded, with
+ * per-rank host arrays of W device pointers.
+ */
+#define AR_STATIC_QK_MAX_T 4096
+#define AR_STATIC_QK_MAX_W 16
+AR_API int ar_group_qk_norm_sharded_static(int W, const void *const *qkv, const void *q_weight,
+                                           const void *k_weight, void *const *q_out,
+                                           void *const *k_out, int64_t T, int64_t q_size,
+                                           int64_t kv_size, float eps, int dtype,
+                                           cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -621,3 +621,96 @@ int ar_group_qk_norm_sharded(ar_comm *g, const void *const *qkv, const void *q_w
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free group QK-norm.  Some callers cannot call cudaMalloc: a
+// plugin that only receives buffers from its host application, an engine
+// that reserved all free device memory when it started (so any further
+// allocation fails), or code that must not take the implicit device-wide
+// synchronisation cudaMalloc may perform.  ar_group_qk_norm_sharded_static
+// runs the same kernel as ar_group_qk_norm_sharded, with the W ranks'
+// exchange regions in this file-scope array instead of a communicator's
+// allocation.  Every GPU that loads the library holds the array until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kStaticSlot = (int64_t)AR_STATIC_QK_MAX_T * 8;       // a token's (q, k) pair: 8 bytes
+constexpr int64_t kStaticRegion = (kSigBytes + 255) / 256 * 256 + 2 * kStaticSlot;
+constexpr int64_t kStaticBytes = kStaticRegion * AR_STATIC_QK_MAX_W;   // about 2 MiB
+
+__device__ __align__(256) uint8_t g_static_qk_scratch[kStaticBytes];
+
+constexpr int kStaticMaxDevices = 64;
+std::once_flag g_static_once[kStaticMaxDevices];
+uint8_t *g_static_ptr[kStaticMaxDevices];
+int g_static_status[kStaticMaxDevices];
+
+// Device address of the array on the current device, looked up once per
+// device (in host code the array's name is only a stand-in, not an address
+// a kernel may use).
+int static_scratch(int dev, uint8_t **out) {
+    if (dev < 0 || dev >= kStaticMaxDevices) return AR_EUNSUPPORTED;
+    std::call_once(g_static_once[dev], [dev] {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_qk_scratch) != cudaSuccess) {
+            (void)cudaGetLastError();
+            g_static_status[dev] = AR_ECUDA;
+            return;
+        }
+        g_static_ptr[dev] = static_cast<uint8_t *>(ptr);
+        g_static_status[dev] = AR_OK;
+    });
+    *out = g_static_ptr[dev];
+    return g_static_status[dev];
+}
+
+}  // namespace
+
+extern "C" int ar_group_qk_norm_sharded_static(int W, const void *const *qkv, const void *q_weight,
+                                               const void *k_weight, void *const *q_out,
+                                               void *const *k_out, int64_t T, int64_t q_size,
+                                               int64_t kv_size, float eps, int dtype,
+                                               cudaStream_t stream) {
+    if (W < 1 || W > AR_STATIC_QK_MAX_W || qkv == nullptr || q_out == nullptr || k_out == nullptr)
+        return AR_EINVAL;
+    if (T < 0) return AR_EINVAL;
+    if (T > AR_STATIC_QK_MAX_T) return AR_EUNSUPPORTED;
+    DevInfo di;
+    int st = device_info(di);
+    if (st != AR_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return AR_ECUDA;
+    uint8_t *base = nullptr;
+    st = static_scratch(dev, &base);
+    if (st != AR_OK) return st;
+    // a communicator description on the stack (nothing allocated) whose W
+    // regions are slices of the array
+    ar_comm g;
+    g.group = true;
+    g.world = W;
+    g.dev = dev;
+    g.sm_count = di.sm_count;
+    g.max_elems = 4 * (int64_t)AR_STATIC_QK_MAX_T;
+    g.part_slot = kStaticSlot;
+    g.gath_slot = 0;
+    g.region_bytes = kStaticRegion;
+    for (int w = 0; w < W; ++w) g.region[w] = base + (int64_t)w * kStaticRegion;
+    g.ready = true;
+    QKCall a = {};
+    for (int r = 0; r < W; ++r) {
+        a.qkv[r] = qkv[r];
+        a.q_out[r] = q_out[r];
+        a.k_out[r] = k_out[r];
+    }
+    if (T == 0) return run_xqk(&g, W, a, q_weight, k_weight, T, q_size, kv_size, eps, dtype, stream);
+    // The array keeps the last call's contents: every call starts from zero
+    // arrival flags and counters in the W regions it uses (stream-ordered
+    // after the previous call on this stream).
+    if (cudaMemset2DAsync(base, (size_t)kStaticRegion, 0, (size_t)kSigBytes, (size_t)W, stream) !=
+        cudaSuccess) {
+        (void)cudaGetLastError();
+        return AR_ECUDA;
+    }
+    return run_xqk(&g, W, a, q_weight, k_weight, T, q_size, kv_size, eps, dtype, stream);
+}
