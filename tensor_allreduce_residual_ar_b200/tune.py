@@ -205,7 +205,9 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--out", default=os.path.join(os.path.dirname(os.path.abspath(__file__)),
                                                   "plan_table.json"))
-    ap.add_argument("--report", default=None)
+    ap.add_argument("--report", default=os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                     "plan_report.jsonl"),
+                    help="per-plan microseconds of every tuned shape (one JSON line per shape)")
     ap.add_argument("--reps", type=int, default=10)
     a = ap.parse_args(argv)
     device = torch.device("cuda", 0)
