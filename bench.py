@@ -750,6 +750,10 @@ def run_launches(args):
     calls = workload_calls(args.workload)
     if args.only_T:
         calls = [c for c in calls if c[2] in args.only_T]
+    if args.force_plan:
+        variant = 2 if args.workload == "qk" else 1 if args.workload == "fp8" else 0
+        if ar.ar_plan_force(variant, args.force_plan) != 0:
+            raise ValueError(f"plan {args.force_plan} is not a plan of the {args.workload} workload")
     bufs = [CallBuffers(c, device) for c in calls]
     for _ in range(args.launches):
         for b in bufs:
@@ -928,6 +932,8 @@ def main(argv=None):
                     help="profiling mode: run every call this many times and exit")
     ap.add_argument("--only-T", type=int, nargs="*", default=None,
                     help="profiling mode: restrict to these T")
+    ap.add_argument("--force-plan", type=int, default=0,
+                    help="profiling mode: run every call with this dispatch plan")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
