@@ -74,11 +74,11 @@ def test_oracle_rows_are_independent():
 
 
 def test_sweep_summary_fields():
-    sweep = {"prefill": [{"T": 8192, "dtype": "bf16", "us": 104.0, "frac_of_measured": 0.98,
+    sweep = {"prefill": [{"T": 8192, "dtype": "bf16", "us": 104.0, "frac_of_peak": 0.98,
                           "frac_of_8TBps": 0.8, "plan": 9}],
-             "decode": [{"T": 1, "dtype": "bf16", "us": 2.5, "frac_of_measured": 0.01,
+             "decode": [{"T": 1, "dtype": "bf16", "us": 2.5, "frac_of_peak": 0.01,
                          "frac_of_8TBps": 0.01, "plan": 4},
-                        {"T": 80, "dtype": "bf16", "us": 4.2, "frac_of_measured": 0.3,
+                        {"T": 80, "dtype": "bf16", "us": 4.2, "frac_of_peak": 0.3,
                          "frac_of_8TBps": 0.27, "plan": 4}]}
     s = bench.sweep_summary(sweep)
     assert s["prefill_T8192"] == [104.0, 0.98, 0.8, 9]
