@@ -240,7 +240,12 @@ typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_v
  *                     asynchronous copies (one per shard row), and whole
  *                     warps normalise one token each from it (falls back to
  *                     QK_PERSIST where two tokens and the weights do not fit
- *                     in shared memory). */
+ *                     in shared memory).
+ *   QK_RING           one token per CTA of at most 256 threads, persistent;
+ *                     each thread keeps its packs of the next five tokens in
+ *                     flight as 16-byte asynchronous copies into a shared-
+ *                     memory ring (falls back to QK_PERSIST for tokens wider
+ *                     than 1024 packs). */
 enum {
     AR_PLAN_AUTO = 0,
     AR_PLAN_ROWC1 = 1,
@@ -259,7 +264,8 @@ enum {
     AR_PLAN_QK_C8 = 14,
     AR_PLAN_QK_PERSIST = 15,
     AR_PLAN_QK_PERSIST256 = 16,
-    AR_PLAN_QK_BULK = 17
+    AR_PLAN_QK_BULK = 17,
+    AR_PLAN_QK_RING = 18
 };
 
 /* The plan a call with these arguments would use (for QK, H = q_size + kv_size

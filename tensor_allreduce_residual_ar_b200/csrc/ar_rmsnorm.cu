@@ -506,6 +506,34 @@ int qk_norm_sharded(const void *const *qkv, const void *q_weight, const void *k_
         }
         plan = AR_PLAN_QK_PERSIST;
     }
+    if (plan == AR_PLAN_QK_RING) {
+        // one token per CTA at a time, every shard of it (at most 256
+        // threads, 1, 2 or 4 packs each), the next tokens' copies in a
+        // shared-memory ring; otherwise the persistent register plan
+        int threads = 0, ppt_idx = 0;
+        if (split_threads(W * (p.qsp + p.ksp), 256, threads, ppt_idx)) {
+            p.C = 1;
+            p.spc = W;
+            static const QKKernel bf[kPptVariants] = {&qk_ring_kernel<__nv_bfloat16, 1>,
+                                                      &qk_ring_kernel<__nv_bfloat16, 2>,
+                                                      &qk_ring_kernel<__nv_bfloat16, 4>};
+            static const QKKernel hf[kPptVariants] = {&qk_ring_kernel<__half, 1>, &qk_ring_kernel<__half, 2>,
+                                                      &qk_ring_kernel<__half, 4>};
+            QKKernel fn = dtype == AR_BF16 ? bf[ppt_idx] : hf[ppt_idx];
+            const int smem = kQKRingStages * (1 << ppt_idx) * threads * 16;
+            int st2 = ensure_smem((const void *)fn, dev, smem);
+            if (st2 != AR_OK) return st2;
+            int occ = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, (size_t)smem) != cudaSuccess ||
+                occ < 1) {
+                (void)cudaGetLastError();
+                occ = 1;
+            }
+            const int64_t cap = (int64_t)di.sm_count * occ;
+            return launch(fn, p, T < cap ? T : cap, 1, threads, stream, (size_t)smem);
+        }
+        plan = AR_PLAN_QK_PERSIST;
+    }
     Geometry g = plan_geometry(plan);
     while (g.C > 1 && W % g.C != 0) g.C /= 2;
     int threads = 0, ppt_idx = 0;

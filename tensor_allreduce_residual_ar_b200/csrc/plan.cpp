@@ -36,7 +36,7 @@ std::atomic<int> g_force[3] = {{0}, {0}, {0}};
 bool is_norm_plan(int id) {
     return id >= AR_PLAN_ROWC1 && id <= AR_PLAN_PERSIST_C2_AHEAD;
 }
-bool is_qk_plan(int id) { return id >= AR_PLAN_QK_C1 && id <= AR_PLAN_QK_BULK; }
+bool is_qk_plan(int id) { return id >= AR_PLAN_QK_C1 && id <= AR_PLAN_QK_RING; }
 
 // Minimal reader for {"entries": [{"key": int, ...}, ...]}: every value must
 // be an integer; unknown keys are errors, so a typo cannot silently drop a
@@ -166,6 +166,7 @@ Geometry plan_geometry(int id) {
     case AR_PLAN_QK_PERSIST: return {1, true, 512, 2};
     case AR_PLAN_QK_PERSIST256: return {1, true, 256, 1};
     case AR_PLAN_QK_BULK: return {1, true, 512, 1};
+    case AR_PLAN_QK_RING: return {1, true, 256, 2};
     default: return {1, false, 512, 1};
     }
 }

@@ -25,7 +25,7 @@ from . import workloads as wl
 
 L2_BYTES = 126 * 1024 * 1024
 NORM_PLANS = (1, 2, 3, 4, 5, 6, 7, 8, 9, 10)
-QK_PLANS = (11, 12, 13, 14, 15, 16, 17)
+QK_PLANS = (11, 12, 13, 14, 15, 16, 17, 18)
 T_MAX = 1 << 40
 
 

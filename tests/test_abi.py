@@ -224,8 +224,8 @@ def test_plan_force(clib):
     assert clib.ar_plan_force(0, 10) == OK          # PERSIST_C2_AHEAD, the last norm plan
     assert clib.ar_plan_force(0, 11) == EINVAL
     assert clib.ar_plan_force(2, 8) == EINVAL
-    assert clib.ar_plan_force(2, 17) == OK          # QK_BULK, the last QK plan
-    assert clib.ar_plan_force(2, 18) == EINVAL
+    assert clib.ar_plan_force(2, 18) == OK          # QK_RING, the last QK plan
+    assert clib.ar_plan_force(2, 19) == EINVAL
     assert clib.ar_plan_force(0, 16) == EINVAL
     assert clib.ar_plan_force(2, 0) == OK
     assert clib.ar_plan_force(0, 0) == OK

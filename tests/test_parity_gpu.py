@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 GUARD = 512
 SENT16 = 0x5A5A
 NORM_PLANS = (1, 2, 3, 4, 5, 6, 7, 8, 9, 10)
-QK_PLANS = (11, 12, 13, 14, 15, 16, 17)
+QK_PLANS = (11, 12, 13, 14, 15, 16, 17, 18)
 TD = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
 
