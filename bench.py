@@ -694,6 +694,10 @@ def tp_arm(ar, device, stream, world, rank, iters=100):
                                                          stream=stream))
             qk.append([T, round(t_fused, 2), round(t_base, 2)])
         status = comm.status()
+        # every rank's last exchange kernel has finished reading the others'
+        # regions before any rank frees its own
+        torch.cuda.synchronize()
+        barrier(device)
     finally:
         comm.close()
     return {"norm_us": rows, "norm_fields": "T, H, one-shot, two-shot, copy + NCCL all_reduce + W=1 "

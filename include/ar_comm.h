@@ -111,7 +111,10 @@ AR_API int ar_comm_open(ar_comm *c, const void *records);
 AR_API int ar_comm_create_group(int world, int64_t max_elems, ar_comm **out);
 
 /* Unmaps peers and frees the region; NULL is a no-op.  Synchronises the
- * communicator's device. */
+ * communicator's device.  Every rank must have finished its calls (its
+ * device synchronised, and the ranks met on the host) before any rank
+ * destroys its communicator: another rank's last kernel may still be reading
+ * this rank's region. */
 AR_API int ar_comm_destroy(ar_comm *c);
 
 /* Limit of one cross-rank wait in nanoseconds (default 2 s; >= 1 ms). */

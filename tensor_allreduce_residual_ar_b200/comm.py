@@ -114,6 +114,10 @@ class _Base:
         B._check("ar_comm_test_withhold", _lib().ar_comm_test_withhold(self._c, int(rank)))
 
     def close(self) -> None:
+        """Free this communicator.  For a multi-process communicator every
+        rank must be done with its calls first (a rank's region may still be
+        read by another rank's last kernel): synchronise and meet the other
+        ranks (e.g. a torch.distributed barrier) before closing."""
         if self._c is not None:
             c, self._c = self._c, None
             B._check("ar_comm_destroy", _lib().ar_comm_destroy(c))
