@@ -621,6 +621,7 @@ def tp_arm(ar, device, stream, world, rank, iters=100):
     import torch.distributed as dist
     from tensor_allreduce_residual_ar_b200 import comm as C
     comm = C.Comm(8192 * 8192, device=device)
+    oneshot_max = comm.tune_oneshot_max()          # the measured crossover, set on the communicator
     rows, worst = [], 0.0
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
@@ -704,6 +705,7 @@ def tp_arm(ar, device, stream, world, rank, iters=100):
                                             "norm (us per call, max over ranks; bf16, one partial per rank)",
             **tp_crossover(rows), "max_rel_vs_nccl_path": round(worst, 5),
             "qk_us": qk, "qk_fields": "T, fused, torch sums + NCCL all_reduce + normalise",
+            "oneshot_max_bytes": oneshot_max, "crossover_us": comm.crossover_us,
             "status": status}
 
 

@@ -271,6 +271,56 @@ class Comm(_Base):
                   B._ptr(residual_out), T, H, 128, float(eps), int(bool(gemma)), B._dtype(weight),
                   _algo(algo), stream=stream)
 
+    def tune_oneshot_max(self, H: int = 8192, Ts=(1, 2, 4, 8, 16, 32, 64, 128, 256, 512),
+                         iters: int = 50, group=None) -> int:
+        """Measure the one-shot / two-shot crossover on these ranks and set it.
+
+        Collective: every rank calls it with the same arguments.  For each T
+        both forms run `iters` times (bf16, [T, H], CUDA events on the current
+        stream, the max over ranks as the time); the largest per-rank size
+        T*H*2 up to which one-shot was faster for every measured T below it
+        becomes ``set_oneshot_max``.  Returns that byte count; the times are
+        kept in ``self.crossover_us`` as [T, one-shot us, two-shot us]."""
+        import torch.distributed as dist
+        dev = self.device
+        use_dist = dist.is_available() and dist.is_initialized() and self.world > 1
+        Tmax = max(Ts)
+        g = torch.Generator(device=dev).manual_seed(1234)
+        part = torch.randn(Tmax, H, generator=g, device=dev).to(torch.bfloat16)
+        res = torch.randn(Tmax, H, generator=g, device=dev).to(torch.bfloat16)
+        w = torch.ones(H, dtype=torch.bfloat16, device=dev)
+        out = torch.empty_like(part)
+        stream = torch.cuda.current_stream(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        rows, limit, still_one = [], 0, True
+        for T in sorted(Ts):
+            us = []
+            for algo in ("oneshot", "twoshot"):
+                call = lambda: self.allreduce_add_rmsnorm(part[:T], res[:T], w, out[:T], None,
+                                                          algo=algo, stream=stream)
+                for _ in range(5):
+                    call()
+                torch.cuda.synchronize(dev)
+                if use_dist:
+                    dist.barrier(group=group)
+                a.record(stream)
+                for _ in range(iters):
+                    call()
+                b.record(stream)
+                b.synchronize()
+                t = torch.tensor([a.elapsed_time(b) * 1e3 / iters], dtype=torch.float64, device=dev)
+                if use_dist:
+                    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+                us.append(float(t.item()))
+            rows.append([T, round(us[0], 3), round(us[1], 3)])
+            if still_one and us[0] <= us[1]:
+                limit = T * H * 2
+            else:
+                still_one = False
+        self.crossover_us = rows
+        self.set_oneshot_max(limit)
+        return limit
+
     def qk_norm_sharded(self, qkv, q_weight, k_weight, q_out, k_out, q_size: int, kv_size: int,
                         eps: float = 1e-6, stream=None):
         """This rank's shard of the sharded QK-norm (q and k normalised over

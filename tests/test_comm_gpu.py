@@ -308,3 +308,20 @@ def test_rank_form_graph_replays_advance_the_epoch(lib):
         assert c.status() == 0
     finally:
         c.close()
+
+
+def test_crossover_tuning_sets_the_communicator(lib):
+    """The collective crossover measurement runs both forms and sets the
+    one-shot limit to a measured size (world size 1 here: both forms are the
+    rank's own sum)."""
+    c = C.Comm(512 * 4096)
+    try:
+        limit = c.tune_oneshot_max(H=4096, Ts=(1, 8, 64, 512), iters=5)
+        assert limit in (0, 1 * 4096 * 2, 8 * 4096 * 2, 64 * 4096 * 2, 512 * 4096 * 2)
+        assert [r[0] for r in c.crossover_us] == [1, 8, 64, 512]
+        assert all(r[1] > 0 and r[2] > 0 for r in c.crossover_us)
+        for T in (1, 8, 64, 512):
+            assert c.algo(T, 4096) == ("oneshot" if T * 4096 * 2 <= limit else "twoshot")
+        assert c.status() == 0
+    finally:
+        c.close()
