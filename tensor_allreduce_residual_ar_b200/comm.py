@@ -86,6 +86,18 @@ def exchange_records(record: bytes, group=None) -> bytes:
     return b"".join(records)
 
 
+def oneshot_limit(rows, H: int) -> int:
+    """From measured [T, one-shot us, two-shot us] rows in increasing T: the
+    per-rank bytes T*H*2 of the largest T up to which one-shot was never
+    slower (0 when two-shot already wins at the smallest T)."""
+    limit = 0
+    for T, one, two in rows:
+        if one > two:
+            break
+        limit = T * H * 2
+    return limit
+
+
 def check_records(blob: bytes, world: int) -> int:
     """The library's consistency check of a gathered record set (host only):
     0 when every rank's record agrees, else an ar_status."""
@@ -292,7 +304,7 @@ class Comm(_Base):
         out = torch.empty_like(part)
         stream = torch.cuda.current_stream(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        rows, limit, still_one = [], 0, True
+        rows = []
         for T in sorted(Ts):
             us = []
             for algo in ("oneshot", "twoshot"):
@@ -313,10 +325,7 @@ class Comm(_Base):
                     dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
                 us.append(float(t.item()))
             rows.append([T, round(us[0], 3), round(us[1], 3)])
-            if still_one and us[0] <= us[1]:
-                limit = T * H * 2
-            else:
-                still_one = False
+        limit = oneshot_limit(rows, H)
         self.crossover_us = rows
         self.set_oneshot_max(limit)
         return limit

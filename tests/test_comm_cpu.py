@@ -125,3 +125,11 @@ def test_rank_that_never_joins_is_an_error_not_a_hang():
     res = _run("absent")
     assert res[1] == "left"
     assert isinstance(res[0], str) and res[0].startswith("error:")
+
+
+def test_oneshot_limit_from_measured_rows():
+    from tensor_allreduce_residual_ar_b200.comm import oneshot_limit
+    rows = [[1, 5.0, 7.0], [8, 6.0, 7.5], [64, 9.0, 8.0], [512, 30.0, 20.0]]
+    assert oneshot_limit(rows, 8192) == 8 * 8192 * 2
+    assert oneshot_limit([[1, 9.0, 8.0], [8, 5.0, 7.0]], 4096) == 0      # first loss ends it
+    assert oneshot_limit([[1, 5.0, 5.0], [2, 5.0, 6.0]], 1024) == 2 * 1024 * 2   # ties go one-shot
