@@ -137,16 +137,25 @@ def time_plan(variant: int, plan: int, sets, reps: int, stream) -> float:
         ar.ar_plan_force(variant, 0)
 
 
+# Token counts measured beyond the workloads' own, so that calls of those
+# shapes at other lengths get a measured plan rather than the neighbouring
+# one's (the prefill shape at decode and long-prefill lengths; QK past 2048
+# tokens, where the register load-ahead plan overtakes the shared-memory ring).
+PREFILL_EXTRA_TS = (16, 256, 2048, 32768)
+QK_EXTRA_TS = (8192, 32768)
+
+
 def default_shapes():
     out = []
     for dt in wl.DECODE.dtypes:
         for T in wl.DECODE.Ts:
             out.append((0, dt, 4, 8192, T, True, True))
     out.append((0, "bf16", 2, 4096, 16, True, True))
-    out.append((0, "bf16", 8, 4096, 8192, True, False))
+    for T in sorted(set(wl.PREFILL.Ts) | set(PREFILL_EXTRA_TS)):
+        out.append((0, "bf16", 8, 4096, T, True, False))
     for T in wl.FP8.Ts:
         out.append((1, "bf16", 4, 5120, T, True, True))
-    for T in wl.QK.Ts:
+    for T in sorted(set(wl.QK.Ts) | set(QK_EXTRA_TS)):
         out.append((2, "bf16", 8, 6144 + 1024, T, 6144, 1024))
     return out
 
