@@ -731,8 +731,9 @@ def run_reference(args):
     el, n, step_bytes = oracle_sample(calls, float("inf"), max_steps=args.steps, row_fraction=frac,
                                       threads=threads)
     value = step_bytes * n / el / 1e9
-    sample = (f"{n} steps of the {args.workload} workload ({len(calls)} calls each, "
-              f"first {frac:.3g} of each call's rows), C fp64 on {threads} threads")
+    rows = "every row of each call" if frac >= 1.0 else f"the first {frac * 100:.3g}% of each call's rows"
+    sample = (f"{n} steps of the {args.workload} workload ({len(calls)} call(s) each, {rows}), "
+              f"C fp64 on {threads} threads")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "GB/s",
             "n_gpus": world, "steps": n, "warmup": args.warmup, "ms_per_step": round(el / n * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
