@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill|decode|tiny|fp8|qk] [--no-sweep]
+    python bench.py --sweep-only --sweep qk [--sweep-T 1 64 2048 ...] [--force-plan P]
 
 One step = one pass over every call of the chosen workload, each call
 through the C ABI, the whole step captured once in a CUDA graph per rotating
@@ -51,13 +52,15 @@ NOMINAL_HBM_GBS = 8000.0
 # workloads as lists of calls
 # ----------------------------------------------------------------------------
 
-def workload_calls(name: str):
+def workload_calls(name: str, Ts=None):
+    """Every call of a workload: (kind, workload, T, dtype), over the
+    workload's token counts or the given ones."""
     from tensor_allreduce_residual_ar_b200 import workloads as wl
     if name in ("tiny", "decode", "prefill", "fp8"):
         w = wl.WORKLOADS[name]
-        return [("norm", w, T, dt) for dt in w.dtypes for T in w.Ts]
+        return [("norm", w, T, dt) for dt in w.dtypes for T in (Ts or w.Ts)]
     if name == "qk":
-        return [("qk", wl.QK, T, "bf16") for T in wl.QK.Ts]
+        return [("qk", wl.QK, T, "bf16") for T in (Ts or wl.QK.Ts)]
     raise ValueError(name)
 
 
@@ -351,7 +354,7 @@ def time_graphs(graphs, n, stream, label=None):
     return start.elapsed_time(end) / 1e3
 
 
-def per_call_sweep(ar, device, stream, names, reps=20):
+def per_call_sweep(ar, device, stream, names, reps=20, Ts=None):
     """Per-call device time of every (workload, T, dtype): one graph holding
     the call once per rotating buffer set, replayed `reps` times."""
     import torch
@@ -359,7 +362,7 @@ def per_call_sweep(ar, device, stream, names, reps=20):
     peak, _ = load_peaks()
     for name in names:
         rows = []
-        for call in workload_calls(name):
+        for call in workload_calls(name, Ts):
             nbytes = call_bytes(call)
             R = min(rotation_sets(nbytes), 2048)
             base = CallBuffers(call, device)
@@ -865,18 +868,7 @@ def run_ours(args):
     if rank != 0:
         return 0
     if not args.no_sweep:
-        names = ["tiny", "decode", "qk", "fp8", "prefill"] if args.sweep == "all" else \
-            [n for n in args.sweep.split(",") if n]
-        sweep = per_call_sweep(ar, device, stream, names)
-        for name, rows in sweep.items():
-            for r in rows:
-                hot = f" (hot L2 {r['us_hot_l2']} us)" if "us_hot_l2" in r else ""
-                print(f"sweep {name} T={r['T']} {r['dtype']}: {r['us']} us{hot}, {r['GBps']} GB/s, "
-                      f"{r['frac_of_peak']} of the {peak_src} peak, {r['frac_of_8TBps']} of 8 TB/s, "
-                      f"plan {r['plan']}", flush=True)
-        if args.sweep_out:
-            with open(args.sweep_out, "w") as f:
-                json.dump(sweep, f, indent=1)
+        sweep = run_sweep(ar, device, stream, args, peak_src)
         line["sweep_summary"] = sweep_summary(sweep, peak_src)
     if world == 1 and not args.no_cpu_baseline:
         cpu = host_cpu()
@@ -892,6 +884,47 @@ def run_ours(args):
                       f"on {threads} threads over row blocks; value_1_thread: one step on the "
                       f"first 1/{max(1, threads)} of the rows, one thread"}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def sweep_names(args):
+    return ["tiny", "decode", "qk", "fp8", "prefill"] if args.sweep == "all" else \
+        [n for n in args.sweep.split(",") if n]
+
+
+def run_sweep(ar, device, stream, args, peak_src):
+    """The per-call sweep, printed as text lines (and written as JSON with
+    --sweep-out)."""
+    sweep = per_call_sweep(ar, device, stream, sweep_names(args), Ts=args.sweep_T)
+    for name, rows in sweep.items():
+        for r in rows:
+            hot = f" (hot L2 {r['us_hot_l2']} us)" if "us_hot_l2" in r else ""
+            print(f"sweep {name} T={r['T']} {r['dtype']}: {r['us']} us{hot}, {r['GBps']} GB/s, "
+                  f"{r['frac_of_peak']} of the {peak_src} peak, {r['frac_of_8TBps']} of 8 TB/s, "
+                  f"plan {r['plan']}", flush=True)
+    if args.sweep_out:
+        with open(args.sweep_out, "w") as f:
+            json.dump(sweep, f, indent=1)
+    return sweep
+
+
+def run_sweep_only(args):
+    """Sweep mode: only the per-call sweep of the --sweep workloads, at the
+    --sweep-T token counts if given, with --force-plan applied to every call
+    of the workloads' variant if given; one GPU, nothing else timed."""
+    import torch
+    import tensor_allreduce_residual_ar_b200 as ar
+    device = torch.device("cuda", dist_env()[2])
+    torch.cuda.set_device(device)
+    ar.load_library()
+    _, peak_src = load_peaks()
+    if args.force_plan:
+        for name in sweep_names(args):
+            variant = 2 if name == "qk" else 1 if name == "fp8" else 0
+            if ar.ar_plan_force(variant, args.force_plan) != 0:
+                raise ValueError(f"plan {args.force_plan} is not a plan of the {name} workload")
+    stream = torch.cuda.Stream(device)
+    run_sweep(ar, device, stream, args, peak_src)
     return 0
 
 
@@ -930,6 +963,10 @@ def main(argv=None):
     ap.add_argument("--sweep", default="all", help="workloads for the per-call sweep (comma list or all)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--sweep-out", default=None, help="also write the full sweep as JSON here")
+    ap.add_argument("--sweep-only", action="store_true",
+                    help="run only the per-call sweep (with --sweep-T, --force-plan) and exit")
+    ap.add_argument("--sweep-T", type=int, nargs="*", default=None,
+                    help="token counts for the sweep instead of each workload's own")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tp", action="store_true", help="N > 1: skip the multi-GPU exchange arm")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -940,7 +977,7 @@ def main(argv=None):
     ap.add_argument("--only-T", type=int, nargs="*", default=None,
                     help="profiling mode: restrict to these T")
     ap.add_argument("--force-plan", type=int, default=0,
-                    help="profiling mode: run every call with this dispatch plan")
+                    help="profiling and sweep modes: run every call with this dispatch plan")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -948,6 +985,8 @@ def main(argv=None):
         return run_reference(args)
     if args.launches:
         return run_launches(args)
+    if args.sweep_only:
+        return run_sweep_only(args)
     return run_ours(args)
 
 

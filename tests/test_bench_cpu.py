@@ -92,3 +92,12 @@ def test_tp_crossover():
     assert c == {"twoshot_beats_oneshot_from_T": 256, "nccl_beats_fused_from_T": 8192}
     assert bench.tp_crossover(rows[:2]) == {"twoshot_beats_oneshot_from_T": None,
                                             "nccl_beats_fused_from_T": None}
+
+
+def test_workload_calls_take_other_token_counts():
+    import bench
+    base = bench.workload_calls("qk")
+    assert [c[2] for c in base] == [1, 64, 2048]
+    assert [c[2] for c in bench.workload_calls("qk", [4096, 8192])] == [4096, 8192]
+    dec = bench.workload_calls("decode", [3])
+    assert [(c[2], c[3]) for c in dec] == [(3, "bf16"), (3, "fp16")]
