@@ -142,7 +142,7 @@ def time_plan(variant: int, plan: int, sets, reps: int, stream) -> float:
 # one's (the prefill shape at decode and long-prefill lengths; QK past 2048
 # tokens, where the register load-ahead plan overtakes the shared-memory ring).
 PREFILL_EXTRA_TS = (16, 256, 2048, 32768)
-QK_EXTRA_TS = (8192, 32768)
+QK_EXTRA_TS = (4096, 8192, 32768)
 
 
 def default_shapes():
