@@ -241,11 +241,13 @@ typedef enum { AR_VARIANT_NORM = 0, AR_VARIANT_FP8 = 1, AR_VARIANT_QK = 2 } ar_v
  *                     warps normalise one token each from it (falls back to
  *                     QK_PERSIST where two tokens and the weights do not fit
  *                     in shared memory).
- *   QK_RING           one token per CTA of at most 256 threads, persistent;
- *                     each thread keeps its packs of the next five tokens in
- *                     flight as 16-byte asynchronous copies into a shared-
- *                     memory ring (falls back to QK_PERSIST for tokens wider
- *                     than 1024 packs). */
+ *   QK_RING           every shard of a token in one CTA of at most 256
+ *                     threads, persistent, two tokens per step (one
+ *                     reduction for their four sums of squares); each thread
+ *                     keeps its packs of the four tokens after the current
+ *                     pair in flight as 16-byte asynchronous copies into a
+ *                     six-token shared-memory ring (falls back to QK_PERSIST
+ *                     for tokens wider than 1024 packs). */
 enum {
     AR_PLAN_AUTO = 0,
     AR_PLAN_ROWC1 = 1,
