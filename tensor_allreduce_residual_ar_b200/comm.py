@@ -8,6 +8,9 @@
 ``CommGroup``  W ranks inside this process on one GPU, every rank's part run
                in one cooperative launch: the same exchange protocol and
                kernels on one device (tests, single-GPU emulation).
+``register``   an integer id for a ``Comm``, by which the torch operators
+               ``torch.ops.ar_b200.tp_*`` and the graph rewrite's all-reduce
+               marker name it (an operator schema cannot carry the object).
 
 Argument marshalling only: tensors are checked (type, dtype, shape,
 contiguity, device) before anything reaches the library, and every step of
@@ -102,6 +105,34 @@ def check_records(blob: bytes, world: int) -> int:
     """The library's consistency check of a gathered record set (host only):
     0 when every rank's record agrees, else an ar_status."""
     return _lib().ar_comm_check_handles(ctypes.c_char_p(blob), world)
+
+
+_REGISTRY: dict = {}
+_NEXT_ID = [1]
+
+
+def register(c: "Comm") -> int:
+    """Register a rank-form communicator; returns the id the tensor-parallel
+    operators and ``fx_patterns.tp_all_reduce_reference`` take.  Every rank
+    registers its own communicator; ids are per process (ranks registering
+    in the same order get the same ids).  Valid until ``unregister``."""
+    if not isinstance(c, Comm):
+        raise TypeError("only a rank-form Comm can be registered")
+    i = _NEXT_ID[0]
+    _NEXT_ID[0] += 1
+    _REGISTRY[i] = c
+    return i
+
+
+def unregister(comm_id: int) -> None:
+    _REGISTRY.pop(int(comm_id), None)
+
+
+def lookup(comm_id: int):
+    c = _REGISTRY.get(int(comm_id))
+    if c is None:
+        raise ValueError(f"no communicator is registered as {comm_id}")
+    return c
 
 
 class _Base:
@@ -231,6 +262,7 @@ class Comm(_Base):
             self.rank, self.world = 0, 1      # no process group: a single rank
         else:
             raise RuntimeError("a process group was given but torch.distributed is not initialised")
+        self.group = group
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
             else torch.device(device)
         lib = _lib()

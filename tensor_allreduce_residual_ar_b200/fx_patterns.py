@@ -19,6 +19,15 @@ graphs):
     y  = rms_norm(r, (H,), weight, eps)      # or rms_norm(r, (H,), None, eps) * (1 + w)
     q, scales = quant_fp8_group_reference(y) # optional, per-group FP8
 
+and the tensor-parallel form of the same sites, where each rank holds one
+partial and the all-reduce crosses GPUs (the pages' own setting):
+
+    s  = tp_all_reduce_reference(p, comm)    # comm: a ``comm.register`` id
+    ...                                      # then as above
+
+which is rewritten to ``torch.ops.ar_b200.tp_*`` (the all-reduce pulled
+over the communicator inside the fused kernel).
+
 ``fuse_allreduce_rmsnorm(gm)`` rewrites every match in place and returns the
 count per form.  Reading of the pages where they are silent: for
 ``a + b`` feeding the norm, a side that is itself an addition used only there
@@ -60,8 +69,24 @@ def all_reduce_sum_reference(partials):
     return out
 
 
+def tp_all_reduce_reference(x: torch.Tensor, comm: int) -> torch.Tensor:
+    """The tensor-parallel all-reduce (sum) of this rank's partial over the
+    ranks of the communicator registered as `comm`, as the unfused program
+    writes it: a copy, all-reduced through torch.distributed over the
+    communicator's process group (at world size 1, the copy).  A traced
+    graph keeps it as one node."""
+    from . import comm as C
+    c = C.lookup(comm)
+    out = x.clone()
+    if c.world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(out, group=c.group)
+    return out
+
+
 torch.fx.wrap("quant_fp8_group_reference")
 torch.fx.wrap("all_reduce_sum_reference")
+torch.fx.wrap("tp_all_reduce_reference")
 
 _ADDS = {operator.add, torch.add, torch.ops.aten.add.Tensor}
 _NORMS = {F.rms_norm, torch.rms_norm, torch.ops.aten.rms_norm.default}
@@ -143,24 +168,36 @@ def _is_marked_sum(n) -> bool:
         and all(isinstance(a, fx.Node) for a in n.args[0])
 
 
+def _is_tp_sum(n) -> bool:
+    return isinstance(n, fx.Node) and n.op == "call_function" and n.target is tp_all_reduce_reference \
+        and len(n.args) == 2 and isinstance(n.args[0], fx.Node) and isinstance(n.args[1], int) \
+        and not n.kwargs
+
+
 def _split_sum(x: fx.Node):
-    """(partials, residual or None) for the norm's input, or None."""
+    """(partials, residual or None, communicator id or None) for the norm's
+    input, or None."""
     if _is_marked_sum(x):
-        return list(x.args[0]), None
+        return list(x.args[0]), None, None
+    if _is_tp_sum(x):
+        return [x.args[0]], None, x.args[1]
     if not _is_add(x):
         return None
     a, b = x.args
     for s, res in ((a, b), (b, a)):
+        if _is_tp_sum(s) and len(_data_users(s)) == 1 and isinstance(res, fx.Node):
+            return [s.args[0]], res, s.args[1]
+    for s, res in ((a, b), (b, a)):
         if _is_marked_sum(s) and len(_data_users(s)) == 1 and isinstance(res, fx.Node):
-            return list(s.args[0]), res
+            return list(s.args[0]), res, None
     for s, res in ((a, b), (b, a)):
         if _is_add(s) and len(_data_users(s)) == 1 and isinstance(res, fx.Node):
             parts = _leaves(s)
             if parts and len(parts) >= 2:
-                return parts, res
+                return parts, res, None
     parts = _leaves(x)
     if parts and len(parts) >= 2:
-        return parts, None
+        return parts, None, None
     return None
 
 
@@ -182,9 +219,10 @@ def _erase_dead(graph: fx.Graph, nodes):
 def fuse_allreduce_rmsnorm(gm: fx.GraphModule) -> dict:
     """Rewrite every recognised subgraph of ``gm`` to the fused operators.
     Returns the number of rewrites per form: "two_output", "out_only",
-    "no_residual" (counted in addition to the first two), "fp8", "gemma"."""
+    "no_residual" (counted in addition to the first two), "fp8", "gemma",
+    and "tp" (the tensor-parallel ones among them)."""
     graph = gm.graph
-    counts = {"two_output": 0, "out_only": 0, "no_residual": 0, "fp8": 0, "gemma": 0}
+    counts = {"two_output": 0, "out_only": 0, "no_residual": 0, "fp8": 0, "gemma": 0, "tp": 0}
     for node in list(graph.nodes):
         if node.graph is not graph:
             continue
@@ -195,7 +233,12 @@ def fuse_allreduce_rmsnorm(gm: fx.GraphModule) -> dict:
         split = _split_sum(x) if isinstance(x, fx.Node) else None
         if split is None:
             continue
-        parts, residual = split
+        parts, residual, comm = split
+        tp = comm is not None
+        # the fused operators' leading arguments: the W partials, or this
+        # rank's partial; the communicator id goes last
+        lead = parts[0] if tp else list(parts)
+        tail = (comm,) if tp else ()
         # the residual result (r = x) is live if anything other than the
         # norm reads its data
         r_live = any(u is not node for u in _data_users(x))
@@ -212,8 +255,8 @@ def fuse_allreduce_rmsnorm(gm: fx.GraphModule) -> dict:
             continue
         with graph.inserting_before(anchor.next):
             if quant:
-                fused = graph.call_function(torch.ops.ar_b200.add_rmsnorm_fp8_group.default,
-                                            (list(parts), residual, weight, eps, gemma))
+                op = torch.ops.ar_b200.tp_add_rmsnorm_fp8_group if tp else torch.ops.ar_b200.add_rmsnorm_fp8_group
+                fused = graph.call_function(op.default, (lead, residual, weight, eps, gemma) + tail)
                 q_ = graph.call_function(operator.getitem, (fused, 0))
                 s_ = graph.call_function(operator.getitem, (fused, 1))
                 y_ = graph.call_function(operator.getitem, (fused, 2))
@@ -226,16 +269,16 @@ def fuse_allreduce_rmsnorm(gm: fx.GraphModule) -> dict:
                 y_node.replace_all_uses_with(y_)
                 counts["fp8"] += 1
             elif r_live:
-                fused = graph.call_function(torch.ops.ar_b200.add_rmsnorm.default,
-                                            (list(parts), residual, weight, eps, gemma))
+                op = torch.ops.ar_b200.tp_add_rmsnorm if tp else torch.ops.ar_b200.add_rmsnorm
+                fused = graph.call_function(op.default, (lead, residual, weight, eps, gemma) + tail)
                 y_ = graph.call_function(operator.getitem, (fused, 0))
                 r_ = graph.call_function(operator.getitem, (fused, 1))
                 y_node.replace_all_uses_with(y_)
                 graph_nodes_to_drop = []
                 counts["two_output"] += 1
             else:
-                y_ = graph.call_function(torch.ops.ar_b200.add_rmsnorm_out_only.default,
-                                         (list(parts), residual, weight, eps, gemma))
+                op = torch.ops.ar_b200.tp_add_rmsnorm_out_only if tp else torch.ops.ar_b200.add_rmsnorm_out_only
+                y_ = graph.call_function(op.default, (lead, residual, weight, eps, gemma) + tail)
                 r_ = None
                 y_node.replace_all_uses_with(y_)
                 graph_nodes_to_drop = []
@@ -249,10 +292,11 @@ def fuse_allreduce_rmsnorm(gm: fx.GraphModule) -> dict:
                     u.replace_input_with(x, parts[0])
         counts["no_residual"] += residual is None
         counts["gemma"] += gemma
+        counts["tp"] += tp
         sum_tree, stack = [], [x]
         while stack:
             n = stack.pop()
-            if (_is_add(n) or _is_marked_sum(n)) and n not in parts:
+            if (_is_add(n) or _is_marked_sum(n) or _is_tp_sum(n)) and n not in parts:
                 sum_tree.append(n)
                 stack += [a for a in n.all_input_nodes]
         # the norm's shape argument (getattr / getitem / size of r)

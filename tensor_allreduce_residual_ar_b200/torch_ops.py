@@ -7,6 +7,16 @@
     torch.ops.ar_b200.qk_norm_sharded(qkv, q_weight, k_weight, q_size, kv_size, eps)
         -> (q_out, k_out)
 
+The tensor-parallel form, one partial per rank and a communicator
+registered with ``comm.register`` (its id is the last argument):
+
+    torch.ops.ar_b200.tp_add_rmsnorm(partial, residual, weight, eps, gemma, comm) -> (y, residual_out)
+    torch.ops.ar_b200.tp_add_rmsnorm_out_only(partial, residual, weight, eps, gemma, comm) -> y
+    torch.ops.ar_b200.tp_add_rmsnorm_fp8_group(partial, residual, weight, eps, gemma, comm)
+        -> (q, scales, y, residual_out)
+
+They are collective: every rank calls them in the same order.
+
 They let torch programs use the fused step as one operator: outputs are
 allocated on the inputs' device by torch's caching allocator and computed by
 the library's kernels on the current stream, so the calls can be captured in
@@ -128,3 +138,68 @@ def _qk_norm_sharded_fake(qkv, q_weight, k_weight, q_size, kv_size, eps):
     x, qs, ks = _check_qk(qkv, q_weight, k_weight, q_size, kv_size)
     lead = x.shape[:-1]
     return ([x.new_empty((*lead, qs)) for _ in qkv], [x.new_empty((*lead, ks)) for _ in qkv])
+
+
+# ---------------------------------------------------------------------------
+# tensor-parallel form: this rank's partial, all-reduced over the ranks of a
+# registered communicator inside the fused call
+# ---------------------------------------------------------------------------
+
+def _comm(comm: int):
+    from . import comm as C
+    return C.lookup(comm)
+
+
+@torch.library.custom_op("ar_b200::tp_add_rmsnorm", mutates_args=(), device_types="cuda")
+def tp_add_rmsnorm(partial: torch.Tensor, residual: torch.Tensor | None, weight: torch.Tensor,
+                   eps: float, gemma: bool, comm: int) -> tuple[torch.Tensor, torch.Tensor]:
+    x, _ = _check_norm([partial], residual, weight)
+    y, r = torch.empty_like(x), torch.empty_like(x)
+    _comm(comm).allreduce_add_rmsnorm(partial, residual, weight, y, r, eps=eps, gemma=gemma)
+    return y, r
+
+
+@tp_add_rmsnorm.register_fake
+def _tp_add_rmsnorm_fake(partial, residual, weight, eps, gemma, comm):
+    x, _ = _check_norm([partial], residual, weight)
+    return torch.empty_like(x), torch.empty_like(x)
+
+
+@torch.library.custom_op("ar_b200::tp_add_rmsnorm_out_only", mutates_args=(), device_types="cuda")
+def tp_add_rmsnorm_out_only(partial: torch.Tensor, residual: torch.Tensor | None, weight: torch.Tensor,
+                            eps: float, gemma: bool, comm: int) -> torch.Tensor:
+    x, _ = _check_norm([partial], residual, weight)
+    y = torch.empty_like(x)
+    _comm(comm).allreduce_add_rmsnorm(partial, residual, weight, y, None, eps=eps, gemma=gemma)
+    return y
+
+
+@tp_add_rmsnorm_out_only.register_fake
+def _tp_add_rmsnorm_out_only_fake(partial, residual, weight, eps, gemma, comm):
+    x, _ = _check_norm([partial], residual, weight)
+    return torch.empty_like(x)
+
+
+@torch.library.custom_op("ar_b200::tp_add_rmsnorm_fp8_group", mutates_args=(), device_types="cuda")
+def tp_add_rmsnorm_fp8_group(partial: torch.Tensor, residual: torch.Tensor | None, weight: torch.Tensor,
+                             eps: float, gemma: bool,
+                             comm: int) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+    x, H = _check_norm([partial], residual, weight)
+    if H % 128 != 0:
+        raise ValueError("H must be a multiple of the group size 128")
+    q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty((*x.shape[:-1], H // 128), dtype=torch.float32, device=x.device)
+    y, r = torch.empty_like(x), torch.empty_like(x)
+    _comm(comm).allreduce_add_rmsnorm_quant_fp8_group(partial, residual, weight, q, s, out_y=y,
+                                                      residual_out=r, eps=eps, gemma=gemma)
+    return q, s, y, r
+
+
+@tp_add_rmsnorm_fp8_group.register_fake
+def _tp_add_rmsnorm_fp8_group_fake(partial, residual, weight, eps, gemma, comm):
+    x, H = _check_norm([partial], residual, weight)
+    if H % 128 != 0:
+        raise ValueError("H must be a multiple of the group size 128")
+    return (torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device),
+            torch.empty((*x.shape[:-1], H // 128), dtype=torch.float32, device=x.device),
+            torch.empty_like(x), torch.empty_like(x))

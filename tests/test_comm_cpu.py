@@ -100,6 +100,49 @@ def _worker(rank, world, port, mode, out):
             dist.destroy_process_group()
 
 
+def _marker_worker(rank, world, port, out):
+    import datetime
+    import sys
+    import types
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from tensor_allreduce_residual_ar_b200 import comm as C
+    from tensor_allreduce_residual_ar_b200 import fx_patterns as FX
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=30))
+    try:
+        # the marker needs only the communicator's world size and group
+        C._REGISTRY[5] = types.SimpleNamespace(world=world, group=None)
+        x = torch.full((3, 8), float(rank + 1))
+        y = FX.tp_all_reduce_reference(x, 5)
+        out.put((rank, (float(x[0, 0]), y.tolist())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tensor_parallel_marker_all_reduces_over_the_group():
+    """The unfused program's all-reduce marker sums the ranks' partials
+    through torch.distributed (gloo, world size 2) and leaves its input
+    untouched."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_marker_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    for r in range(world):
+        x0, y = res[r]
+        assert x0 == r + 1
+        assert y == [[3.0] * 8] * 3
+
+
 def _run(mode):
     world, port = 2, _free_port()
     ctx = mp.get_context("spawn")

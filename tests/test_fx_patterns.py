@@ -70,6 +70,52 @@ class TwoLayers(torch.nn.Module):
         return y2
 
 
+COMM = 7      # a communicator id as the traced programs carry it (registered only on the GPU)
+
+
+class TpTwoOutput(torch.nn.Module):
+    def forward(self, p, res, w):
+        r = FX.tp_all_reduce_reference(p, COMM) + res
+        return F.rms_norm(r, (r.shape[-1],), w, 1e-6), r
+
+
+class TpOutOnly(torch.nn.Module):
+    def forward(self, p, res, w):
+        r = res + FX.tp_all_reduce_reference(p, COMM)
+        return F.rms_norm(r, (r.shape[-1],), w, 1e-5)
+
+
+class TpNoResidual(torch.nn.Module):
+    def forward(self, p, w):
+        s = FX.tp_all_reduce_reference(p, COMM)
+        return F.rms_norm(s, (s.shape[-1],), w, 1e-6)
+
+
+class TpGemma(torch.nn.Module):
+    def forward(self, p, res, w):
+        r = FX.tp_all_reduce_reference(p, COMM) + res
+        return F.rms_norm(r, (r.shape[-1],), None, 1e-6) * (1 + w), r
+
+
+class TpFp8(torch.nn.Module):
+    def forward(self, p, res, w):
+        r = FX.tp_all_reduce_reference(p, COMM) + res
+        y = F.rms_norm(r, (r.shape[-1],), w, 1e-6)
+        q, s = FX.quant_fp8_group_reference(y)
+        return q, s, y, r
+
+
+class TpSumReadElsewhere(torch.nn.Module):
+    """The all-reduced sum is read again besides the residual add: the add +
+    norm is still fused (the sum is not a private intermediate of it, so it
+    stays), exactly like a shared partial sum on one GPU."""
+
+    def forward(self, p, res, w):
+        s = FX.tp_all_reduce_reference(p, COMM)
+        r = s + res
+        return F.rms_norm(r, (r.shape[-1],), w, 1e-6), s * 2
+
+
 class NotASum(torch.nn.Module):
     def forward(self, x, res, w):
         r = x * res
@@ -106,7 +152,7 @@ def fuse(mod):
 ])
 def test_each_form_fires_once(mod, want, op):
     gm, c = fuse(mod)
-    full = {"two_output": 0, "out_only": 0, "no_residual": 0, "fp8": 0, "gemma": 0, **want}
+    full = {"two_output": 0, "out_only": 0, "no_residual": 0, "fp8": 0, "gemma": 0, "tp": 0, **want}
     assert c == full
     ops = fused_ops(gm)
     assert [str(t).split(".")[1] for t in ops] == [op]
@@ -114,6 +160,34 @@ def test_each_form_fires_once(mod, want, op):
     assert not any(t in FX._NORMS for t in left), "the unfused norm is gone"
     assert FX.quant_fp8_group_reference not in left and FX.all_reduce_sum_reference not in left
     assert not any(t in FX._ADDS for t in left), "the partial sum and the residual add are gone"
+
+
+@pytest.mark.parametrize("mod,want,op", [
+    (TpTwoOutput(), {"two_output": 1}, "tp_add_rmsnorm"),
+    (TpOutOnly(), {"out_only": 1}, "tp_add_rmsnorm_out_only"),
+    (TpNoResidual(), {"out_only": 1, "no_residual": 1}, "tp_add_rmsnorm_out_only"),
+    (TpGemma(), {"two_output": 1, "gemma": 1}, "tp_add_rmsnorm"),
+    (TpFp8(), {"fp8": 1}, "tp_add_rmsnorm_fp8_group"),
+])
+def test_tensor_parallel_forms_route_to_the_communicator(mod, want, op):
+    gm, c = fuse(mod)
+    full = {"two_output": 0, "out_only": 0, "no_residual": 0, "fp8": 0, "gemma": 0, "tp": 1, **want}
+    assert c == full
+    ops = fused_ops(gm)
+    assert [str(t).split(".")[1] for t in ops] == [op]
+    node = [n for n in gm.graph.nodes if str(n.target).startswith("ar_b200.")][0]
+    assert node.args[-1] == COMM and node.args[0].op == "placeholder"   # this rank's partial, the id
+    left = targets(gm)
+    assert FX.tp_all_reduce_reference not in left
+    assert not any(t in FX._NORMS for t in left)
+
+
+def test_tensor_parallel_sum_read_elsewhere():
+    gm, c = fuse(TpSumReadElsewhere())
+    # the all-reduce is not private to the add + norm: the add is fused as
+    # the sum of two plain terms (s and res) and the all-reduce stays
+    assert c["tp"] == 0 and c["two_output"] + c["out_only"] == 1
+    assert FX.tp_all_reduce_reference in targets(gm)
 
 
 def test_two_layers_chain():
@@ -126,7 +200,7 @@ def test_two_layers_chain():
 def test_unrecognised_graphs_are_left_alone(mod):
     gm, c = fuse(mod)
     before = torch.fx.symbolic_trace(mod)
-    assert c == {"two_output": 0, "out_only": 0, "no_residual": 0, "fp8": 0, "gemma": 0}
+    assert c == {"two_output": 0, "out_only": 0, "no_residual": 0, "fp8": 0, "gemma": 0, "tp": 0}
     assert targets(gm) == targets(before)
 
 
@@ -173,3 +247,48 @@ def test_rewritten_program_matches_oracle(lib, mod_cls, W, has_res):
     P.check_y(P.to_bits(y.contiguous()), o["y"], "bf16")
     if len(outs) > 1:
         P.check_res(P.to_bits(outs[1]), o["r"], "bf16")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mod_cls,has_res", [(TpTwoOutput, True), (TpOutOnly, True), (TpNoResidual, False),
+                                             (TpGemma, True), (TpFp8, True)])
+def test_tensor_parallel_rewrite_matches_oracle(lib, mod_cls, has_res):
+    """The rewritten tensor-parallel programs on a world-size-1 communicator
+    (the all-reduce of one rank's partial is the partial itself) against the
+    oracle; the operator passes torch.library.opcheck."""
+    import parity as P
+    from tensor_allreduce_residual_ar_b200 import comm as C
+    from tensor_allreduce_residual_ar_b200 import workloads as wl
+    T, H = 37, 1024
+    c = C.Comm(T * H)
+    C._REGISTRY[COMM] = c          # the id the traced programs carry
+    try:
+        inp = wl.make_norm_inputs(wl.FP8, T, W=1, H=H, residual=has_res, seed=7300 + has_res)
+        gemma = mod_cls is TpGemma
+        inp.gemma = gemma
+        gm, cnt = fuse(mod_cls())
+        assert cnt["tp"] == 1
+        args = [inp.partials[0].cuda()] + ([inp.residual.cuda()] if has_res else []) + [inp.weight.cuda()]
+        eps = {TpOutOnly: wl.eps32(1e-5)}.get(mod_cls, wl.eps32(1e-6))
+        ref = wl.NormInputs(inp.partials, inp.residual if has_res else None, inp.weight, T, H, 1, "bf16",
+                            eps, gemma, True)
+        o = P.oracle_norm(ref)
+        for prog in (gm,):
+            out = prog(*args)
+            torch.cuda.synchronize()
+            outs = out if isinstance(out, tuple) else (out,)
+            if mod_cls is TpFp8:
+                q, s, y, r = outs
+                P.check_fp8(q.view(torch.uint8).cpu().numpy(), s.cpu().numpy(), o["y"])
+                P.check_y(P.to_bits(y), o["y"], "bf16")
+                P.check_res(P.to_bits(r), o["r"], "bf16")
+                continue
+            P.check_y(P.to_bits(outs[0].contiguous()), o["y"], "bf16")
+            if len(outs) > 1:
+                P.check_res(P.to_bits(outs[1]), o["r"], "bf16")
+        if mod_cls is TpTwoOutput:
+            torch.library.opcheck(torch.ops.ar_b200.tp_add_rmsnorm.default,
+                                  (args[0], args[1], args[2], 1e-6, False, COMM))
+    finally:
+        C._REGISTRY.pop(COMM, None)
+        c.close()

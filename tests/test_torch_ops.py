@@ -35,6 +35,24 @@ def test_fake_shapes_norm_and_fp8():
         assert y3.shape == r3.shape == (2, 3, 5120)
 
 
+def test_tensor_parallel_ops_schemas_and_fake_shapes():
+    s = str(OPS.tp_add_rmsnorm.default._schema)
+    assert "Tensor partial, Tensor? residual, Tensor weight, float eps, bool gemma, SymInt comm" in s
+    assert s.endswith("-> (Tensor, Tensor)")
+    assert str(OPS.tp_add_rmsnorm_out_only.default._schema).endswith("-> Tensor")
+    assert str(OPS.tp_add_rmsnorm_fp8_group.default._schema).endswith("-> (Tensor, Tensor, Tensor, Tensor)")
+    with FakeTensorMode():
+        p = torch.empty(5, 5120, dtype=torch.bfloat16, device="cuda")
+        w = torch.empty(5120, dtype=torch.bfloat16, device="cuda")
+        y, r = OPS.tp_add_rmsnorm(p, p, w, 1e-6, False, 3)
+        assert y.shape == r.shape == (5, 5120)
+        assert OPS.tp_add_rmsnorm_out_only(p, None, w, 1e-6, True, 3).shape == (5, 5120)
+        q, sc, y2, r2 = OPS.tp_add_rmsnorm_fp8_group(p, p, w, 1e-6, False, 3)
+        assert q.dtype == torch.float8_e4m3fn and sc.shape == (5, 40)
+        with pytest.raises(ValueError):
+            OPS.tp_add_rmsnorm(p, p[:, :4096], w, 1e-6, False, 3)
+
+
 def test_fake_shapes_qk():
     with FakeTensorMode():
         qkv = [torch.empty(7, 768 + 256, dtype=torch.float16, device="cuda") for _ in range(8)]
