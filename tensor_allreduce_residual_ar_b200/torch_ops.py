@@ -14,6 +14,8 @@ registered with ``comm.register`` (its id is the last argument):
     torch.ops.ar_b200.tp_add_rmsnorm_out_only(partial, residual, weight, eps, gemma, comm) -> y
     torch.ops.ar_b200.tp_add_rmsnorm_fp8_group(partial, residual, weight, eps, gemma, comm)
         -> (q, scales, y, residual_out)
+    torch.ops.ar_b200.tp_qk_norm_sharded(qkv, q_weight, k_weight, q_size, kv_size, eps, comm)
+        -> (q_out, k_out)        # this rank's shard; only per-token sums of squares cross ranks
 
 They are collective: every rank calls them in the same order.
 
@@ -203,3 +205,42 @@ def _tp_add_rmsnorm_fp8_group_fake(partial, residual, weight, eps, gemma, comm):
     return (torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device),
             torch.empty((*x.shape[:-1], H // 128), dtype=torch.float32, device=x.device),
             torch.empty_like(x), torch.empty_like(x))
+
+
+def _check_tp_qk(qkv, q_weight, k_weight, q_size, kv_size, world):
+    if q_size % world or kv_size % world:
+        raise ValueError(f"q_size and kv_size must be multiples of the world size {world}")
+    qs, ks = q_size // world, kv_size // world
+    if qs % 8 or ks % 8:
+        raise ValueError("per-rank q and k widths must be multiples of 8")
+    if qkv.shape[-1] != qs + 2 * ks:
+        raise ValueError("this rank's qkv must be [..., q_size/W + 2*kv_size/W]")
+    if tuple(q_weight.shape) != (q_size,) or tuple(k_weight.shape) != (kv_size,):
+        raise ValueError("q_weight must be [q_size] and k_weight [kv_size]")
+    if qkv.dtype not in _DT or q_weight.dtype != qkv.dtype or k_weight.dtype != qkv.dtype:
+        raise TypeError("bf16 or fp16 tensors of one dtype are supported")
+    return qs, ks
+
+
+@torch.library.custom_op("ar_b200::tp_qk_norm_sharded", mutates_args=(), device_types="cuda")
+def tp_qk_norm_sharded(qkv: torch.Tensor, q_weight: torch.Tensor, k_weight: torch.Tensor, q_size: int,
+                       kv_size: int, eps: float, comm: int) -> tuple[torch.Tensor, torch.Tensor]:
+    c = _comm(comm)
+    qs, ks = _check_tp_qk(qkv, q_weight, k_weight, q_size, kv_size, c.world)
+    lead = qkv.shape[:-1]
+    qo = torch.empty((*lead, qs), dtype=qkv.dtype, device=qkv.device)
+    ko = torch.empty((*lead, ks), dtype=qkv.dtype, device=qkv.device)
+    c.qk_norm_sharded(qkv, q_weight, k_weight, qo, ko, q_size, kv_size, eps=eps)
+    return qo, ko
+
+
+@tp_qk_norm_sharded.register_fake
+def _tp_qk_norm_sharded_fake(qkv, q_weight, k_weight, q_size, kv_size, eps, comm):
+    # the world size is the communicator's; the shard's width fixes it
+    row = qkv.shape[-1]
+    world = (q_size + 2 * kv_size) // row if row else 0
+    if world < 1 or world * row != q_size + 2 * kv_size:
+        raise ValueError("qkv's width must be (q_size + 2*kv_size) / W for the communicator's W")
+    qs, ks = _check_tp_qk(qkv, q_weight, k_weight, q_size, kv_size, world)
+    lead = qkv.shape[:-1]
+    return qkv.new_empty((*lead, qs)), qkv.new_empty((*lead, ks))

@@ -292,3 +292,26 @@ def test_tensor_parallel_rewrite_matches_oracle(lib, mod_cls, has_res):
     finally:
         C._REGISTRY.pop(COMM, None)
         c.close()
+
+
+@pytest.mark.gpu
+def test_tensor_parallel_qk_operator_matches_oracle(lib):
+    """torch.ops.ar_b200.tp_qk_norm_sharded on a world-size-1 communicator
+    (the rank's shard is the whole q and k) against the oracle."""
+    import parity as P
+    from tensor_allreduce_residual_ar_b200 import comm as C
+    from tensor_allreduce_residual_ar_b200 import workloads as wl
+    T = 33
+    inp = wl.make_qk_inputs(wl.QK, T, "bf16", W=1, q_size=6144, kv_size=1024, seed=7400)
+    c = C.Comm(T * (6144 + 2 * 1024))
+    cid = C.register(c)
+    try:
+        qo, ko = torch.ops.ar_b200.tp_qk_norm_sharded(inp.qkv[0].cuda(), inp.q_weight.cuda(),
+                                                      inp.k_weight.cuda(), 6144, 1024, 1e-6, cid)
+        torch.cuda.synchronize()
+        q64, k64 = P.oracle_qk(inp)
+        P.check_y(P.to_bits(qo), q64[0], "bf16")
+        P.check_y(P.to_bits(ko), k64[0], "bf16")
+    finally:
+        C.unregister(cid)
+        c.close()

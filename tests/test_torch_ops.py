@@ -51,6 +51,12 @@ def test_tensor_parallel_ops_schemas_and_fake_shapes():
         assert q.dtype == torch.float8_e4m3fn and sc.shape == (5, 40)
         with pytest.raises(ValueError):
             OPS.tp_add_rmsnorm(p, p[:, :4096], w, 1e-6, False, 3)
+        qkv = torch.empty(9, 768 + 256, dtype=torch.bfloat16, device="cuda")     # W = 8 shard
+        qw = torch.empty(6144, dtype=torch.bfloat16, device="cuda")
+        kw = torch.empty(1024, dtype=torch.bfloat16, device="cuda")
+        qo, ko = OPS.tp_qk_norm_sharded(qkv, qw, kw, 6144, 1024, 1e-6, 3)
+        assert qo.shape == (9, 768) and ko.shape == (9, 128)
+    assert str(OPS.tp_qk_norm_sharded.default._schema).endswith("-> (Tensor, Tensor)")
 
 
 def test_fake_shapes_qk():
