@@ -315,3 +315,41 @@ def test_tensor_parallel_qk_operator_matches_oracle(lib):
     finally:
         C.unregister(cid)
         c.close()
+
+
+@pytest.mark.gpu
+def test_tensor_parallel_operator_in_a_cuda_graph(lib):
+    """The tensor-parallel operator captured in a CUDA graph on a world-size-1
+    communicator: replays give the eager call's bits (new inputs copied into
+    the captured buffers between replays)."""
+    from tensor_allreduce_residual_ar_b200 import comm as C
+    from tensor_allreduce_residual_ar_b200 import workloads as wl
+    T, H = 24, 2048
+    c = C.Comm(T * H)
+    cid = C.register(c)
+    try:
+        ins = [wl.make_norm_inputs(wl.DECODE, T, "bf16", W=1, H=H, seed=7500 + i) for i in range(3)]
+        p = ins[0].partials[0].cuda()
+        res = ins[0].residual.cuda()
+        w = ins[0].weight.cuda()
+        op = torch.ops.ar_b200.tp_add_rmsnorm
+        op(p, res, w, 1e-6, True, cid)                     # first call outside capture
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                y, r = op(p, res, w, 1e-6, True, cid)
+        for inp in ins[1:]:
+            p.copy_(inp.partials[0])
+            res.copy_(inp.residual)
+            g.replay()
+            torch.cuda.synchronize()
+            y0, r0 = op(p.clone(), res.clone(), w, 1e-6, True, cid)
+            torch.cuda.synchronize()
+            assert torch.equal(y.view(torch.int16), y0.view(torch.int16))
+            assert torch.equal(r.view(torch.int16), r0.view(torch.int16))
+        del g
+    finally:
+        C.unregister(cid)
+        c.close()
