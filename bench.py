@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload prefill|decode|tiny|fp8|qk] [--no-sweep]
     python bench.py --sweep-only --sweep qk [--sweep-T 1 64 2048 ...] [--force-plan P]
+    python bench.py --sweep-only --sweep exchange   # the exchange kernels at world size 1
 
 One step = one pass over every call of the chosen workload, each call
 through the C ABI, the whole step captured once in a CUDA graph per rotating
@@ -892,11 +893,76 @@ def sweep_names(args):
         [n for n in args.sweep.split(",") if n]
 
 
+def exchange_sweep(ar, device, stream, Ts=None, reps=20):
+    """The exchange kernels' own cost on one GPU: the rank-form communicator
+    at world size 1 runs the multi-GPU kernels (the partial staged into the
+    communicator's region, the sys-scope flag barrier, then the fused add +
+    norm reading the staged rows), with no NVLink in the path.  Per token
+    count of the decode shape (H = 8192, bf16, residual and residual_out),
+    and the prefill-sized T = 8192 at H = 4096: device time per call of the
+    plain fused call with one partial, of the one-shot and of the two-shot
+    form, each in a CUDA graph over rotating buffer sets as in the sweep."""
+    import torch
+    from tensor_allreduce_residual_ar_b200 import comm as C
+    shapes = [(T, 8192) for T in (Ts or (1, 16, 80, 512))] + ([] if Ts else [(8192, 4096)])
+    rows = []
+    for T, H in shapes:
+        nbytes = T * H * 2 * 4 + H * 2          # partial, residual, y, residual_out
+        R = min(rotation_sets(nbytes), 2048)
+        g = torch.Generator(device=device).manual_seed(4242 + T)
+        w = (torch.randn(H, generator=g, device=device) * 0.1).to(torch.bfloat16)
+        sets = []
+        for _ in range(R):
+            t = [(torch.randn(T, H, generator=g, device=device)).to(torch.bfloat16) for _ in range(2)]
+            sets.append((t[0], t[1], torch.empty_like(t[0]), torch.empty_like(t[0])))
+        comm = C.Comm(T * H, device=device)
+        res = {"T": T, "H": H, "sets": R}
+        try:
+            forms = {
+                "plain": lambda b: ar.ar_add_rmsnorm([b[0]], b[1], w, b[2], b[3], eps=1e-6, gemma=True,
+                                                     stream=stream),
+                "oneshot": lambda b: comm.allreduce_add_rmsnorm(b[0], b[1], w, b[2], b[3], eps=1e-6,
+                                                                gemma=True, algo="oneshot", stream=stream),
+                "twoshot": lambda b: comm.allreduce_add_rmsnorm(b[0], b[1], w, b[2], b[3], eps=1e-6,
+                                                                gemma=True, algo="twoshot", stream=stream),
+            }
+            for name, f in forms.items():
+                with torch.cuda.stream(stream):
+                    f(sets[0])
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    with torch.cuda.graph(graph, stream=stream):
+                        for b in sets:
+                            f(b)
+                time_graphs([graph], 2, stream)
+                sec = time_graphs([graph], reps, stream) / (reps * R)
+                res[name + "_us"] = round(sec * 1e6, 3)
+                del graph
+            torch.cuda.synchronize()
+            if comm.status() != 0:
+                raise RuntimeError("an exchange wait timed out")
+        finally:
+            comm.close()
+        rows.append(res)
+        del sets
+        torch.cuda.empty_cache()
+    return rows
+
+
 def run_sweep(ar, device, stream, args, peak_src):
     """The per-call sweep, printed as text lines (and written as JSON with
     --sweep-out)."""
-    sweep = per_call_sweep(ar, device, stream, sweep_names(args), Ts=args.sweep_T)
+    names = sweep_names(args)
+    sweep = per_call_sweep(ar, device, stream, [n for n in names if n != "exchange"], Ts=args.sweep_T)
+    if "exchange" in names:
+        sweep["exchange"] = exchange_sweep(ar, device, stream, Ts=args.sweep_T)
+        for r in sweep["exchange"]:
+            print(f"sweep exchange T={r['T']} H={r['H']} bf16: plain {r['plain_us']} us, one-shot "
+                  f"{r['oneshot_us']} us, two-shot {r['twoshot_us']} us (world size 1)", flush=True)
     for name, rows in sweep.items():
+        if name == "exchange":
+            continue
         for r in rows:
             hot = f" (hot L2 {r['us_hot_l2']} us)" if "us_hot_l2" in r else ""
             print(f"sweep {name} T={r['T']} {r['dtype']}: {r['us']} us{hot}, {r['GBps']} GB/s, "
