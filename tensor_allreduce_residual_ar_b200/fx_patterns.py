@@ -26,7 +26,9 @@ partial and the all-reduce crosses GPUs (the pages' own setting):
     ...                                      # then as above
 
 which is rewritten to ``torch.ops.ar_b200.tp_*`` (the all-reduce pulled
-over the communicator inside the fused kernel).
+over the communicator inside the fused kernel).  The marker is matched as
+the one node ``symbolic_trace`` keeps for it; torch's functional collectives
+in an aten-level graph are not matched.
 
 ``fuse_allreduce_rmsnorm(gm)`` rewrites every match in place and returns the
 count per form.  Reading of the pages where they are silent: for
