@@ -190,6 +190,32 @@ def test_tensor_parallel_sum_read_elsewhere():
     assert FX.tp_all_reduce_reference in targets(gm)
 
 
+class TpTwoSublayers(torch.nn.Module):
+    """A tensor-parallel decoder layer's two norm sites: the attention
+    output's all-reduce + residual + RMSNorm (two outputs: the residual
+    stream continues), then the MLP's (output only, the layer's last)."""
+
+    def __init__(self, H=64):
+        super().__init__()
+        self.proj_a = torch.nn.Linear(H, H, bias=False)
+        self.proj_b = torch.nn.Linear(H, H, bias=False)
+
+    def forward(self, x, res, w1, w2):
+        r1 = FX.tp_all_reduce_reference(self.proj_a(x), COMM) + res
+        y1 = F.rms_norm(r1, (r1.shape[-1],), w1, 1e-6)
+        r2 = FX.tp_all_reduce_reference(self.proj_b(y1), COMM) + r1
+        return F.rms_norm(r2, (r2.shape[-1],), w2, 1e-6)
+
+
+def test_tensor_parallel_two_sublayers():
+    gm, c = fuse(TpTwoSublayers())
+    assert c["tp"] == 2 and c["two_output"] == 1 and c["out_only"] == 1
+    assert [str(t).split(".")[1] for t in fused_ops(gm)] == ["tp_add_rmsnorm", "tp_add_rmsnorm_out_only"]
+    assert FX.tp_all_reduce_reference not in targets(gm)
+    # the projections (call_module) are untouched
+    assert sum(n.op == "call_module" for n in gm.graph.nodes) == 2
+
+
 def test_two_layers_chain():
     gm, c = fuse(TwoLayers())
     assert c["two_output"] == 1 and c["out_only"] == 1
