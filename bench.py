@@ -750,11 +750,44 @@ def run_reference(args):
     return 0
 
 
+def run_exchange_launches(args):
+    """Profiling mode for the multi-GPU kernels: the world-size-1 rank-form
+    call (decode shape H = 8192, bf16, residual and residual_out) in the
+    --exchange form, `--launches` times per --only-T token count (default 1),
+    plain stream launches."""
+    import torch
+    import tensor_allreduce_residual_ar_b200 as ar
+    from tensor_allreduce_residual_ar_b200 import comm as C
+    device = torch.device("cuda", dist_env()[2])
+    torch.cuda.set_device(device)
+    ar.load_library()
+    H = 8192
+    Ts = args.only_T or [1]
+    comm = C.Comm(max(Ts) * H, device=device)
+    try:
+        g = torch.Generator(device=device).manual_seed(4243)
+        w = (torch.randn(H, generator=g, device=device) * 0.1).to(torch.bfloat16)
+        for T in Ts:
+            p_, r_ = [torch.randn(T, H, generator=g, device=device).to(torch.bfloat16) for _ in range(2)]
+            y, ro = torch.empty_like(p_), torch.empty_like(p_)
+            for _ in range(args.launches):
+                comm.allreduce_add_rmsnorm(p_, r_, w, y, ro, eps=1e-6, gemma=True, algo=args.exchange)
+        torch.cuda.synchronize()
+        if comm.status() != 0:
+            raise RuntimeError("an exchange wait timed out")
+    finally:
+        comm.close()
+    print(json.dumps({"launches": args.launches * len(Ts), "exchange": args.exchange, "T": Ts, "H": H}))
+    return 0
+
+
 def run_launches(args):
     """Profiling mode: every call of the workload `--launches` times, plain
     stream launches (no graph, no timing), for a profiler to capture."""
     import torch
     import tensor_allreduce_residual_ar_b200 as ar
+    if args.exchange:
+        return run_exchange_launches(args)
     device = torch.device("cuda", dist_env()[2])
     torch.cuda.set_device(device)
     ar.load_library()
@@ -1040,6 +1073,8 @@ def main(argv=None):
                     help="untimed load before the timed region (clocks settle, sampler runs)")
     ap.add_argument("--launches", type=int, default=0,
                     help="profiling mode: run every call this many times and exit")
+    ap.add_argument("--exchange", choices=["oneshot", "twoshot"], default=None,
+                    help="profiling mode: the multi-GPU kernel at world size 1 instead of a workload")
     ap.add_argument("--only-T", type=int, nargs="*", default=None,
                     help="profiling mode: restrict to these T")
     ap.add_argument("--force-plan", type=int, default=0,
