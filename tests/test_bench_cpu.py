@@ -101,3 +101,20 @@ def test_workload_calls_take_other_token_counts():
     assert [c[2] for c in bench.workload_calls("qk", [4096, 8192])] == [4096, 8192]
     dec = bench.workload_calls("decode", [3])
     assert [(c[2], c[3]) for c in dec] == [(3, "bf16"), (3, "fp16")]
+
+
+def test_reference_arm_line():
+    """The reference arm (the CPU oracle on the host cores) prints its JSON
+    line with the same metric and unit, no GPU involved."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "3", "--warmup", "3"],
+                       cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][-1])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "GB/s" and d["steps"] == 3
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
