@@ -980,6 +980,51 @@ def exchange_sweep(ar, device, stream, Ts=None, reps=20):
         rows.append(res)
         del sets
         torch.cuda.empty_cache()
+    # the sharded QK-norm's exchange (only each token's two sums of squares
+    # cross ranks) at world size 1, against the plain call with one shard
+    for T in (Ts or (1, 64, 2048)):
+        q_size, kv_size = 6144, 1024
+        row = q_size + 2 * kv_size
+        nbytes = T * (q_size + kv_size) * 2 * 2
+        R = min(rotation_sets(nbytes), 2048)
+        g = torch.Generator(device=device).manual_seed(4343 + T)
+        qw = (1 + 0.1 * torch.randn(q_size, generator=g, device=device)).to(torch.bfloat16)
+        kw = (1 + 0.1 * torch.randn(kv_size, generator=g, device=device)).to(torch.bfloat16)
+        sets = []
+        for _ in range(R):
+            x = torch.randn(T, row, generator=g, device=device).to(torch.bfloat16)
+            sets.append((x, torch.empty(T, q_size, dtype=torch.bfloat16, device=device),
+                         torch.empty(T, kv_size, dtype=torch.bfloat16, device=device)))
+        comm = C.Comm(T * row, device=device)
+        res = {"T": T, "H": q_size + kv_size, "sets": R, "qk": True}
+        try:
+            forms = {
+                "plain": lambda b: ar.qk_norm_sharded([b[0]], qw, kw, [b[1]], [b[2]], q_size, kv_size,
+                                                      eps=1e-6, stream=stream),
+                "exchange": lambda b: comm.qk_norm_sharded(b[0], qw, kw, b[1], b[2], q_size, kv_size,
+                                                           eps=1e-6, stream=stream),
+            }
+            for name, f in forms.items():
+                with torch.cuda.stream(stream):
+                    f(sets[0])
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    with torch.cuda.graph(graph, stream=stream):
+                        for b in sets:
+                            f(b)
+                time_graphs([graph], 2, stream)
+                sec = time_graphs([graph], reps, stream) / (reps * R)
+                res[name + "_us"] = round(sec * 1e6, 3)
+                del graph
+            torch.cuda.synchronize()
+            if comm.status() != 0:
+                raise RuntimeError("an exchange wait timed out")
+        finally:
+            comm.close()
+        rows.append(res)
+        del sets
+        torch.cuda.empty_cache()
     return rows
 
 
@@ -991,6 +1036,10 @@ def run_sweep(ar, device, stream, args, peak_src):
     if "exchange" in names:
         sweep["exchange"] = exchange_sweep(ar, device, stream, Ts=args.sweep_T)
         for r in sweep["exchange"]:
+            if r.get("qk"):
+                print(f"sweep exchange qk T={r['T']} q+kv={r['H']} bf16: plain {r['plain_us']} us, "
+                      f"exchange {r['exchange_us']} us (world size 1)", flush=True)
+                continue
             print(f"sweep exchange T={r['T']} H={r['H']} bf16: plain {r['plain_us']} us, one-shot "
                   f"{r['oneshot_us']} us, two-shot {r['twoshot_us']} us (world size 1)", flush=True)
     for name, rows in sweep.items():
