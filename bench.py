@@ -162,6 +162,8 @@ _REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_
 class ClockSampler:
     def __init__(self, device_index: int, period_s: float = 0.005):
         self.samples = []
+        self.mem_samples = []
+        self.power_w = []
         self.reasons = 0
         self.max_mhz = None
         self._stop = threading.Event()
@@ -187,6 +189,11 @@ class ClockSampler:
                 self.reasons |= int(get_reasons(self._h))
             except Exception:
                 pass
+            try:   # context for a number taken under the power cap (read-only)
+                self.mem_samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_MEM))
+                self.power_w.append(nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0)
+            except Exception:
+                pass
             time.sleep(self.period)
 
     def __enter__(self):
@@ -204,8 +211,13 @@ class ClockSampler:
         if self._nv is None:
             return {"unavailable": getattr(self, "error", "no NVML")}
         names = [n for b, n in _REASONS.items() if self.reasons & b and b != 0x1]
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names}
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names}
+        if self.mem_samples:
+            out["mem_mhz"] = statistics.median(self.mem_samples)
+        if self.power_w:
+            out["power_w"] = round(statistics.median(self.power_w), 1)
+        return out
 
 
 # ----------------------------------------------------------------------------
